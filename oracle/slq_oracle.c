@@ -1,0 +1,330 @@
+/*
+ * slq_oracle.c -- plain, slow, scalar CPU oracle for the SLQ weight format.
+ *
+ * TEST INFRASTRUCTURE ONLY (see slq_oracle.h).  Each function states the
+ * passage it follows.  Nothing here is blocked, fused or reordered: every
+ * loop is the definition written out, one element at a time.
+ *
+ * Where the pages are silent the library fixes a reading, and this file
+ * follows the same reading, stated where it is used:
+ *   - scale is rounded to fp16 first and the encode uses that stored scale;
+ *   - a group whose min equals its max is widened to include 0;
+ *   - an all-zero group stores scale 1.0, zero 0, codes 0;
+ *   - a nonzero fp32 scale that rounds to fp16 zero is stored as 2^-24;
+ *     one that overflows fp16 is stored as 65504 and flagged;
+ *   - codes are packed LSB-first into one bitstream per row, so a group of
+ *     128 codes fills exactly 4*b uint32 words.
+ *
+ * Build: gcc -O2 -fno-fast-math -ffp-contract=off -shared -fPIC.
+ */
+#include "slq_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define GROUP 128
+
+/* ---------------------------------------------------------------------- */
+/* Number formats (IEEE 754 binary16 and bfloat16), written out by hand.   */
+/* ---------------------------------------------------------------------- */
+
+static uint32_t f32_bits(float f) {
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  return u;
+}
+
+static float bits_f32(uint32_t u) {
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+/* Round the integer x right by sh bits, to nearest, ties to even. */
+static uint32_t shift_right_rne(uint32_t x, int sh) {
+  if (sh <= 0) return x;
+  if (sh >= 32) return 0; /* x < 2^24 here, so x / 2^sh < 1/2 */
+  uint32_t q = x >> sh;
+  uint32_t rem = x & ((1u << sh) - 1u);
+  uint32_t half = 1u << (sh - 1);
+  if (rem > half || (rem == half && (q & 1u))) q += 1u;
+  return q;
+}
+
+uint16_t oracle_f32_to_f16_rn(float f) {
+  uint32_t u = f32_bits(f);
+  uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+  uint32_t e = (u >> 23) & 0xFFu;
+  uint32_t m = u & 0x7FFFFFu;
+  if (e == 0xFFu) return (uint16_t)(sign | (m ? 0x7E00u : 0x7C00u));
+  if (e == 0u) return sign; /* |f| < 2^-126: far below half of 2^-24 */
+  int E = (int)e - 127;     /* f = sig * 2^(E - 23) */
+  uint32_t sig = (1u << 23) | m;
+  if (E > 15) return (uint16_t)(sign | 0x7C00u);
+  if (E >= -14) {
+    /* Normal binary16: keep 11 significant bits. */
+    uint32_t r = shift_right_rne(sig, 13);
+    if (r == (1u << 11)) { /* rounding carried into the next binade */
+      r = 1u << 10;
+      E += 1;
+    }
+    if (E > 15) return (uint16_t)(sign | 0x7C00u);
+    return (uint16_t)(sign | ((uint32_t)(E + 15) << 10) | (r - (1u << 10)));
+  }
+  /* Subnormal binary16: count units of 2^-24.  A result of 2^10 units is the
+   * smallest normal, whose bit pattern is the same integer. */
+  uint32_t r = shift_right_rne(sig, -E - 1);
+  return (uint16_t)(sign | r);
+}
+
+double oracle_f16_to_f64(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int e = (h >> 10) & 0x1F;
+  int m = h & 0x3FF;
+  double v;
+  if (e == 0)
+    v = ldexp((double)m, -24);
+  else if (e == 31)
+    v = m ? NAN : INFINITY;
+  else
+    v = ldexp((double)(1024 + m), e - 25);
+  return sign ? -v : v;
+}
+
+float oracle_bf16_to_f32(uint16_t h) { return bits_f32((uint32_t)h << 16); }
+
+/* ---------------------------------------------------------------------- */
+/* Quantize + pack.                                                        */
+/* ---------------------------------------------------------------------- */
+
+/* Write code q (bits wide) at stream bit position pos of one row's words,
+ * least significant bit first: stream bit i is bit (i mod 32) of word i/32. */
+static void put_code(uint32_t *row_words, int64_t pos, int bits, uint32_t q) {
+  int64_t w = pos / 32;
+  int sh = (int)(pos % 32);
+  row_words[w] |= q << sh;
+  if (sh + bits > 32) row_words[w + 1] |= q >> (32 - sh);
+}
+
+uint32_t oracle_code_at(const uint32_t *packed, int64_t K, int bits, int64_t n,
+                        int64_t k) {
+  const uint32_t *row = packed + n * (K * bits / 32);
+  int64_t pos = k * bits;
+  int64_t w = pos / 32;
+  int sh = (int)(pos % 32);
+  uint64_t window = row[w];
+  if (sh + bits > 32) window |= (uint64_t)row[w + 1] << 32;
+  return (uint32_t)((window >> sh) & ((1u << bits) - 1u));
+}
+
+/*
+ * One group of 128 weights along K.  The pages fix: asymmetric integer grid,
+ * group size 128, b in {2..8} (gist.science "The SLQ Pipeline"; GitHub README
+ * "Pipeline"), round to nearest (RTN).  The library's format definition fixes
+ * the arithmetic in binary32:
+ *   scale = (max - min) / (2^b - 1), zero = clamp(rne(-min / scale)),
+ *   q = clamp(rne(w / scale) + zero), codes in [0, 2^b - 1].
+ */
+static void quantize_group(const uint16_t *src, int bits, uint16_t *s16_out,
+                           uint8_t *z_out, uint32_t *codes, uint32_t *flags) {
+  float w[GROUP];
+  int nonfinite = 0;
+  for (int k = 0; k < GROUP; ++k) {
+    w[k] = oracle_bf16_to_f32(src[k]);
+    if (!isfinite(w[k])) nonfinite = 1;
+  }
+  if (nonfinite && flags) *flags |= ORACLE_FLAG_NONFINITE;
+
+  /* Group statistics: min and max in binary32 (exact). */
+  float mn = w[0], mx = w[0];
+  for (int k = 1; k < GROUP; ++k) {
+    if (w[k] < mn) mn = w[k];
+    if (w[k] > mx) mx = w[k];
+  }
+
+  /* Reading: a constant group is widened to include 0, so that it
+   * reconstructs to (about) itself instead of dividing by a zero range. */
+  float lo = mn, hi = mx;
+  if (hi == lo) {
+    if (lo > 0.0f) lo = 0.0f;
+    if (hi < 0.0f) hi = 0.0f;
+  }
+
+  const float maxq = (float)((1 << bits) - 1);
+  float s32 = (hi - lo) / maxq; /* one binary32 subtraction, one IEEE division */
+
+  /* Reading: the scale is stored in fp16 and the encode uses the stored
+   * value, so the reconstruction bound holds for what the GEMM reads. */
+  uint16_t s16;
+  if (s32 == 0.0f) {
+    s16 = 0x3C00u; /* all-zero group: scale 1.0 */
+  } else {
+    s16 = oracle_f32_to_f16_rn(s32);
+    if ((s16 & 0x7FFFu) == 0u) {
+      s16 = 0x0001u; /* nonzero scale below fp16 range: 2^-24 */
+    } else if (s16 == 0x7C00u) {
+      s16 = 0x7BFFu; /* beyond fp16 range: 65504, flagged */
+      if (flags) *flags |= ORACLE_FLAG_SCALE_OVERFLOW;
+    }
+  }
+  const float s = (float)oracle_f16_to_f64(s16);
+
+  /* Zero point: rne(-min / scale), clamped to the code range. */
+  float zf = rintf(-lo / s);
+  if (zf != zf || zf < 0.0f) zf = 0.0f;
+  if (zf > maxq) zf = maxq;
+
+  /* Codes: rne(w / scale) + zero, clamped to the code range.  The sum is
+   * taken in binary32: it is exact whenever the result is inside the range. */
+  for (int k = 0; k < GROUP; ++k) {
+    float v = rintf(w[k] / s) + zf;
+    if (v != v || v < 0.0f) v = 0.0f;
+    if (v > maxq) v = maxq;
+    codes[k] = (uint32_t)v;
+  }
+  *s16_out = s16;
+  *z_out = (uint8_t)zf;
+}
+
+int oracle_quantize(const uint16_t *w_bf16, int64_t N, int64_t K, int bits,
+                    uint32_t *packed, uint16_t *scales_f16, uint8_t *zeros,
+                    uint32_t *flags) {
+  if (bits < 2 || bits > 8 || N < 0 || K < 0 || K % GROUP != 0) return -1;
+  const int64_t G = K / GROUP;
+  const int64_t words_per_row = K * bits / 32;
+  memset(packed, 0, (size_t)(N * words_per_row) * sizeof(uint32_t));
+  uint32_t codes[GROUP];
+  for (int64_t n = 0; n < N; ++n) {
+    uint32_t *row_words = packed + n * words_per_row;
+    for (int64_t g = 0; g < G; ++g) {
+      quantize_group(w_bf16 + n * K + g * GROUP, bits, &scales_f16[n * G + g],
+                     &zeros[n * G + g], codes, flags);
+      for (int j = 0; j < GROUP; ++j)
+        put_code(row_words, (g * GROUP + j) * bits, bits, codes[j]);
+    }
+  }
+  return 0;
+}
+
+/* ---------------------------------------------------------------------- */
+/* Dequantize and GEMM (weight-only, bf16 activations).                    */
+/* ---------------------------------------------------------------------- */
+
+/* w' = s * (q - z): the fake-quantized weight the pages store (GitHub README,
+ * "1. Quantize" and "4. Build and serve a checkpoint").  Exact in binary64. */
+static void dequantize_row(const uint32_t *packed, const uint16_t *scales_f16,
+                           const uint8_t *zeros, int64_t K, int bits, int64_t n,
+                           double *out) {
+  const int64_t G = K / GROUP;
+  for (int64_t k = 0; k < K; ++k) {
+    int64_t g = k / GROUP;
+    double s = oracle_f16_to_f64(scales_f16[n * G + g]);
+    double q = (double)oracle_code_at(packed, K, bits, n, k);
+    double z = (double)zeros[n * G + g];
+    out[k] = s * (q - z);
+  }
+}
+
+int oracle_dequantize(const uint32_t *packed, const uint16_t *scales_f16,
+                      const uint8_t *zeros, int64_t N, int64_t K, int bits,
+                      double *w_out) {
+  if (bits < 2 || bits > 8 || K % GROUP != 0) return -1;
+  for (int64_t n = 0; n < N; ++n)
+    dequantize_row(packed, scales_f16, zeros, K, bits, n, w_out + n * K);
+  return 0;
+}
+
+/* Y = X W^T with w' as above: y[m, n] = sum_k x[m, k] * w'[n, k], binary64,
+ * k ascending.  This is the weight-only linear layer that the serving
+ * kernels compute (gist.science "Inference Speedup"; GitHub README intro). */
+int oracle_gemm(const uint16_t *x_bf16, const int64_t *rows, int64_t n_rows,
+                int64_t N, int64_t K, int bits, const uint32_t *packed,
+                const uint16_t *scales_f16, const uint8_t *zeros, double *y) {
+  if (bits < 2 || bits > 8 || K % GROUP != 0) return -1;
+  /* Widen the sampled rows of X once (bf16 -> double is exact). */
+  double *xd = (double *)malloc((size_t)(n_rows * K) * sizeof(double));
+  double *wrow = (double *)malloc((size_t)K * sizeof(double));
+  if (!xd || !wrow) {
+    free(xd);
+    free(wrow);
+    return -2;
+  }
+  for (int64_t i = 0; i < n_rows; ++i) {
+    int64_t m = rows ? rows[i] : i;
+    for (int64_t k = 0; k < K; ++k)
+      xd[i * K + k] = (double)oracle_bf16_to_f32(x_bf16[m * K + k]);
+  }
+  for (int64_t n = 0; n < N; ++n) {
+    dequantize_row(packed, scales_f16, zeros, K, bits, n, wrow);
+    for (int64_t i = 0; i < n_rows; ++i) {
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k) acc += xd[i * K + k] * wrow[k];
+      y[i * N + n] = acc;
+    }
+  }
+  free(xd);
+  free(wrow);
+  return 0;
+}
+
+/* ---------------------------------------------------------------------- */
+/* EAR and KL between two softmaxed logit rows.                            */
+/* ---------------------------------------------------------------------- */
+
+/* log sum_v exp(u_v), shifted by the maximum so no term overflows. */
+static double logsumexp(const double *u, int64_t V) {
+  double mx = u[0];
+  for (int64_t v = 1; v < V; ++v)
+    if (u[v] > mx) mx = u[v];
+  if (isinf(mx)) return mx;
+  double sum = 0.0;
+  for (int64_t v = 0; v < V; ++v) sum += exp(u[v] - mx);
+  return mx + log(sum);
+}
+
+/*
+ * For one token: p = softmax(a / tau) (reference model), q = softmax(b / tau)
+ * (quantized model).  EAR = sum_v min(p_v, q_v), the probability that the two
+ * models agree under the optimal coupling (gist.science "Fidelity Metrics";
+ * reddit abstract).  The pages' evaluation restricts it to the top-K tokens;
+ * this is the full-vocabulary case, K = V.  KL(p || q) = sum_v p_v (log p_v -
+ * log q_v) in nats (gist.science "Fidelity Metrics", Task-Lossless search
+ * signal).  log p_v is taken as the log-softmax a_v / tau - logsumexp, so a
+ * p_v that underflows to 0 contributes 0 * finite = 0.
+ */
+int oracle_ear_kl(const uint16_t *a_bf16, const uint16_t *b_bf16,
+                  const int64_t *rows, int64_t n_rows, int64_t V, double tau,
+                  double *ear, double *kl) {
+  if (V < 1 || !(tau > 0.0) || isinf(tau)) return -1;
+  double *x = (double *)malloc((size_t)V * sizeof(double));
+  double *y = (double *)malloc((size_t)V * sizeof(double));
+  if (!x || !y) {
+    free(x);
+    free(y);
+    return -2;
+  }
+  for (int64_t i = 0; i < n_rows; ++i) {
+    int64_t t = rows ? rows[i] : i;
+    for (int64_t v = 0; v < V; ++v) {
+      x[v] = (double)oracle_bf16_to_f32(a_bf16[t * V + v]) / tau;
+      y[v] = (double)oracle_bf16_to_f32(b_bf16[t * V + v]) / tau;
+    }
+    double la = logsumexp(x, V);
+    double lb = logsumexp(y, V);
+    double e = 0.0, d = 0.0;
+    for (int64_t v = 0; v < V; ++v) {
+      double log_p = x[v] - la;
+      double log_q = y[v] - lb;
+      double p = exp(log_p);
+      double q = exp(log_q);
+      e += (p < q) ? p : q;
+      d += p * (log_p - log_q);
+    }
+    ear[i] = e;
+    kl[i] = d;
+  }
+  free(x);
+  free(y);
+  return 0;
+}
