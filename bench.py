@@ -1,0 +1,564 @@
+#!/usr/bin/env python
+"""Benchmark of the SLQ weight-format hot path on B200 (one JSON line).
+
+Headline workload: a Qwen3-8B-shaped decoder block at decode batch sizes --
+hidden 4096, q/o 4096x4096 at 5 bits, k/v 1024x4096 at 8 bits, gate/up
+12288x4096 and down 4096x12288 at 4 bits (asymmetric INT, group 128), X bf16
+~ N(0,1) at M in {1, 4, 16}.  One step = the 7 dequantize-GEMMs of the block
+at each of the three M (21 launches, replayed as one CUDA graph).  The metric
+is packed-weight bytes streamed per second (codes + fp16 scales + uint8
+zeros), whole job over all ranks.
+
+The same line reports the other rows of the hot path, each timed with CUDA
+events on its own stream: quantize+pack of the block's weights, the decode
+sweep N=K=8192 at every b, the tiled GEMM at prefill sizes, and EAR/KL over
+[4096 x 151936] logits.  Inputs are seeded synthetic stand-ins for the
+pages' models (no checkpoints or datasets here).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl slq|reference]
+
+--impl reference times the CPU oracle (the plain reference implementation
+of the same arithmetic) on a bounded sample of the same workload, on the
+host cores, and reports the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+GROUP = 128
+L2_BYTES = 126 * 2**20
+
+# Qwen3-8B-shaped block: (name, N, K, bits)
+QWEN3_8B_BLOCK = [("q", 4096, 4096, 5), ("k", 1024, 4096, 8), ("v", 1024, 4096, 8),
+                  ("o", 4096, 4096, 5), ("gate", 12288, 4096, 4), ("up", 12288, 4096, 4),
+                  ("down", 4096, 12288, 4)]
+DECODE_MS = (1, 4, 16)
+METRIC = "W{2-8}A16 GEMM weight GB/s (% HBM peak) & TFLOP/s per b and M; EAR/KL GB/s"
+
+
+def weight_bytes(N, K, bits):
+    return N * K * bits // 8 + N * (K // GROUP) * 3
+
+
+BLOCK_BYTES = sum(weight_bytes(N, K, b) for _, N, K, b in QWEN3_8B_BLOCK)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ----------------------------------------------------------------------------
+# Clock sampling (nvidia-smi) during the timed region
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# CUDA events as graph nodes (cudaEventRecordExternal) for per-launch timing
+# ----------------------------------------------------------------------------
+class GraphEvents:
+    """Event-record nodes inside a captured graph, read after replay."""
+
+    def __init__(self, n: int):
+        import nvidia.cuda_runtime as cr
+        path = os.path.join(list(cr.__path__)[0], "lib", "libcudart.so.12")
+        self.rt = ctypes.CDLL(path)
+        self.events = []
+        for _ in range(n):
+            ev = ctypes.c_void_p()
+            if self.rt.cudaEventCreate(ctypes.byref(ev)) != 0:
+                raise RuntimeError("cudaEventCreate failed")
+            self.events.append(ev)
+
+    def record(self, i: int, stream_handle: int):
+        rc = self.rt.cudaEventRecordWithFlags(self.events[i], ctypes.c_void_p(stream_handle), 1)
+        if rc != 0:
+            raise RuntimeError(f"cudaEventRecordWithFlags failed ({rc})")
+
+    def elapsed_ms(self, i: int, j: int) -> float:
+        ms = ctypes.c_float()
+        rc = self.rt.cudaEventElapsedTime(ctypes.byref(ms), self.events[i], self.events[j])
+        if rc != 0:
+            raise RuntimeError(f"cudaEventElapsedTime failed ({rc})")
+        return ms.value
+
+
+# ----------------------------------------------------------------------------
+# The SLQ arm
+# ----------------------------------------------------------------------------
+def run_slq(args, rank, world, local_rank):
+    import torch
+    import synth
+    import weight_only_mixed_b200 as slq
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    hbm_peak, tc_peak, tc_peak_sus, peak_kind = load_peaks()
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+    sh = stream.cuda_stream
+
+    # ---- setup (untimed): quantize the block's weights, rotated copies -------
+    R = max(2, int(np.ceil(4 * L2_BYTES / BLOCK_BYTES)))
+    layers = []  # layers[r][i] = QuantizedWeight
+    for r in range(R):
+        copy = []
+        for i, (name, N, K, b) in enumerate(QWEN3_8B_BLOCK):
+            W = synth.weights_torch(N, K, seed=synth.SEED_WEIGHTS + 10 * i + 1000 * r + rank, device=dev)
+            copy.append(slq.quantize(W, b))
+            del W
+        layers.append(copy)
+    X = {M: [synth.activations_torch(M, K, seed=synth.SEED_X + 10 * i + M, device=dev)
+             for i, (_, N, K, b) in enumerate(QWEN3_8B_BLOCK)] for M in DECODE_MS}
+    Y = {M: [torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+             for (_, N, K, b) in QWEN3_8B_BLOCK] for M in DECODE_MS}
+    torch.cuda.synchronize()
+
+    n_launch = len(DECODE_MS) * len(QWEN3_8B_BLOCK)
+    try:
+        gev = [GraphEvents(n_launch + 1) for _ in range(R)]
+    except Exception:
+        gev = None
+
+    def step_body(r, ev=None):
+        k = 0
+        for M in DECODE_MS:
+            for i in range(len(QWEN3_8B_BLOCK)):
+                if ev is not None:
+                    ev.record(k, sh)
+                slq.gemm(X[M][i], layers[r][i], out=Y[M][i], stream=stream)
+                k += 1
+        if ev is not None:
+            ev.record(k, sh)
+
+    # Warm up eagerly once (device attributes, first launches), then capture.
+    step_body(0)
+    torch.cuda.synchronize()
+    graphs = []
+    for r in range(R):
+        g = torch.cuda.CUDAGraph()
+        try:
+            with torch.cuda.graph(g, stream=stream):
+                step_body(r, gev[r] if gev else None)
+        except Exception:
+            gev = None
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step_body(r)
+        graphs.append(g)
+    torch.cuda.synchronize()
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+    for s in range(args.warmup):
+        graphs[s % R].replay()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))
+    clocks.start()
+    time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    reps = max(1, args.repeat)
+    t0.record(stream)
+    for s in range(args.steps * reps):
+        graphs[s % R].replay()
+    t1.record(stream)
+    t1.synchronize()
+    ms_total = t0.elapsed_time(t1)
+    clk = clocks.stop()
+    ms_step = ms_total / (args.steps * reps)
+    if dist:
+        t = torch.tensor([ms_step], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+        dist.barrier()
+
+    value = world * 3 * BLOCK_BYTES / (ms_step * 1e-3) / 1e9  # GB/s, whole job
+
+    # Per-launch durations of the decode kernel from the last replay of each
+    # graph inside the timed region.
+    per_m = {}
+    kernel_ms = None
+    if gev is not None and args.steps * reps >= R:
+        tot_bytes, tot_ms = 0.0, 0.0
+        for r in range(R):
+            k = 0
+            for M in DECODE_MS:
+                for i, (name, N, K, b) in enumerate(QWEN3_8B_BLOCK):
+                    d = gev[r].elapsed_ms(k, k + 1)
+                    wb = weight_bytes(N, K, b)
+                    per_m.setdefault(M, [0.0, 0.0])
+                    per_m[M][0] += wb
+                    per_m[M][1] += d
+                    tot_bytes += wb
+                    tot_ms += d
+                    k += 1
+        kernel_ms = tot_ms / (R * n_launch)
+        achieved = tot_bytes / (tot_ms * 1e-3) / 1e9
+    else:
+        achieved = 3 * BLOCK_BYTES / (ms_step * 1e-3) / 1e9
+    breakdown = {f"M={M}": {"weight_GBps": round(v[0] / (v[1] * 1e-3) / 1e9, 1),
+                            "frac_hbm": round(v[0] / (v[1] * 1e-3) / 1e9 / hbm_peak, 3)}
+                 for M, v in per_m.items()}
+
+    # ---- e2e: public Python API, host buffers, copies inside the timed region
+    Xh = {M: [x.cpu().pin_memory() for x in X[M]] for M in DECODE_MS}
+    Yh = {M: [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in Y[M]] for M in DECODE_MS}
+    Xd = {M: [torch.empty_like(x) for x in X[M]] for M in DECODE_MS}
+    h2d = sum(x.numel() * 2 for M in DECODE_MS for x in X[M])
+    d2h = sum(y.numel() * 2 for M in DECODE_MS for y in Y[M])
+
+    def e2e_step(r):
+        for M in DECODE_MS:
+            for i in range(len(QWEN3_8B_BLOCK)):
+                Xd[M][i].copy_(Xh[M][i], non_blocking=True)
+                slq.gemm(Xd[M][i], layers[r][i], out=Y[M][i], stream=stream)
+                Yh[M][i].copy_(Y[M][i], non_blocking=True)
+        stream.synchronize()
+
+    for s in range(max(1, args.warmup)):
+        e2e_step(s % R)
+    e2e_steps = max(3, args.steps)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in range(e2e_steps):
+        e2e_step(s % R)
+    e1.record(stream)
+    e1.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if dist:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * 3 * BLOCK_BYTES / (e2e_ms * 1e-3) / 1e9
+
+    rows = {}
+    if not args.headline_only:
+        rows = other_rows(args, slq, synth, torch, dev, stream, hbm_peak, tc_peak, rank)
+
+    # free the rotated copies before the CPU baseline
+    del layers, graphs
+    torch.cuda.synchronize()
+
+    out = None
+    if rank == 0:
+        cpu = cpu_baseline(args) if (world == 1 and not args.no_cpu) else None
+        out = {
+            "metric": METRIC,
+            "value": round(value, 1),
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_step, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded skewed-Gaussian weights, N(0,1) activations; no checkpoints)",
+            "config": {
+                "workload": "Qwen3-8B-shaped decoder block decode: q/o 4096x4096 b5, k/v 1024x4096 b8, "
+                            "gate/up 12288x4096 b4, down 4096x12288 b4, asymmetric INT g128; "
+                            "M in {1,4,16}; 21 dequant-GEMM launches per step (one CUDA graph)",
+                "block_weight_bytes": BLOCK_BYTES,
+                "bytes_per_step": 3 * BLOCK_BYTES,
+                "l2": f"inputs larger than L2: {R} rotated weight copies ({R * BLOCK_BYTES / 2**20:.0f} MiB > 126 MiB L2)",
+                "parallelism": f"replicas x{world} (independent layers per rank, no collective)",
+                "repeat": reps,
+            },
+            "roofline": {
+                "bound": "hbm",
+                "kernel": "gemm_decode_kernel (register dequant + mma.m16n8k16, M<=16)",
+                "achieved": round(achieved, 1),
+                "peak": hbm_peak,
+                "unit": "GB/s",
+                "frac": round(achieved / hbm_peak, 4),
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6650 GB/s",
+                "algorithmic_bytes": "N*K*(b/8 + 3/128) per launch (codes + fp16 scale + u8 zero)",
+                "avg_launch_us": round(kernel_ms * 1e3, 3) if kernel_ms else None,
+                "traffic": None,
+                "per_M": breakdown,
+            },
+            "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h,
+                    "how": "public Python API (slq.gemm per projection), X from pinned host, Y back to pinned host, per step"},
+            "gpu_launches": n_launch * args.steps * reps,
+            "clocks": clk,
+            "rows": rows,
+        }
+        if cpu is not None:
+            out["cpu_baseline"] = cpu
+    return out
+
+
+def time_ms(torch, stream, fn, iters, warm=2):
+    for _ in range(warm):
+        fn()
+    stream.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(iters):
+        fn()
+    b.record(stream)
+    b.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+def other_rows(args, slq, synth, torch, dev, stream, hbm_peak, tc_peak, rank):
+    rows = {}
+    # Quantize + pack of the block's 7 weights (reads bf16, writes packed).
+    Ws = [synth.weights_torch(N, K, seed=90 + i, device=dev) for i, (_, N, K, b) in enumerate(QWEN3_8B_BLOCK)]
+    outs = [slq.empty_quantized(N, K, b, dev) for (_, N, K, b) in QWEN3_8B_BLOCK]
+
+    def qstep():
+        for W, q, (_, N, K, b) in zip(Ws, outs, QWEN3_8B_BLOCK):
+            slq.quantize(W, b, out=q, stream=stream)
+
+    ms = time_ms(torch, stream, qstep, 10)
+    qbytes = sum(N * K * 2 + weight_bytes(N, K, b) for _, N, K, b in QWEN3_8B_BLOCK)
+    rows["quantize_block"] = {"GBps": round(qbytes / (ms * 1e-3) / 1e9, 1),
+                              "frac_hbm": round(qbytes / (ms * 1e-3) / 1e9 / hbm_peak, 3),
+                              "us": round(ms * 1e3, 2), "bytes": qbytes}
+    del Ws, outs
+
+    # Decode sweep N = K = 8192 at every b, M in {1, 16}.
+    sweep = {}
+    N = K = 8192
+    for b in range(2, 9):
+        nrot = max(2, int(np.ceil(4 * L2_BYTES / weight_bytes(N, K, b))))
+        qws = [slq.quantize(synth.weights_torch(N, K, seed=700 + b + 10 * r, device=dev), b) for r in range(nrot)]
+        for M in (1, 16):
+            Xs = synth.activations_torch(M, K, seed=800 + M, device=dev)
+            Ys = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            it = [0]
+
+            def f():
+                slq.gemm(Xs, qws[it[0] % nrot], out=Ys, stream=stream)
+                it[0] += 1
+
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for r in range(nrot):
+                    slq.gemm(Xs, qws[r], out=Ys, stream=stream)
+            ms = time_ms(torch, stream, g.replay, 20) / nrot
+            gbps = weight_bytes(N, K, b) / (ms * 1e-3) / 1e9
+            sweep[f"b{b}_M{M}"] = {"GBps": round(gbps, 1), "frac_hbm": round(gbps / hbm_peak, 3),
+                                   "TFLOPs": round(2 * M * N * K / (ms * 1e-3) / 1e12, 2),
+                                   "us": round(ms * 1e3, 2)}
+        del qws
+    rows["decode_sweep_8192"] = sweep
+
+    # EAR / KL over [4096 x 151936] bf16 logits, tau 1.0 and 0.7.
+    T, V = 4096, 151936
+    a, bq = synth.logits_torch(T, V, device=dev)
+    ear = torch.empty(T, dtype=torch.float32, device=dev)
+    kl = torch.empty(T, dtype=torch.float32, device=dev)
+    em = torch.empty((), dtype=torch.float64, device=dev)
+    km = torch.empty((), dtype=torch.float64, device=dev)
+    L = slq.lib()
+    for tau in (1.0, 0.7):
+        def f():
+            rc = L.slq_ear_kl(a.data_ptr(), bq.data_ptr(), T, V, tau, ear.data_ptr(), kl.data_ptr(),
+                              em.data_ptr(), km.data_ptr(), None, stream.cuda_stream)
+            assert rc == 0
+        ms = time_ms(torch, stream, f, 5, warm=1)
+        nbytes = 2 * T * V * 2
+        rows[f"ear_kl_tau{tau}"] = {"GBps": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                                    "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / hbm_peak, 3),
+                                    "us": round(ms * 1e3, 1), "ear_mean": round(em.item(), 6),
+                                    "kl_mean": round(km.item(), 7)}
+    del a, bq
+    return rows
+
+
+# ----------------------------------------------------------------------------
+# CPU baseline / reference arm: the oracle on a bounded sample
+# ----------------------------------------------------------------------------
+def _oracle_sample(rows_per_layer: int):
+    import oracle
+    import synth
+    work = []
+    for i, (name, N, K, b) in enumerate(QWEN3_8B_BLOCK):
+        n = min(N, rows_per_layer)
+        w = synth.weights(n, K, seed=synth.SEED_WEIGHTS + i)
+        packed, scales, zeros, _ = oracle.quantize(w, b)
+        xs = {M: synth.activations(M, K, seed=synth.SEED_X + M + i) for M in DECODE_MS}
+        work.append((n, K, b, packed, scales, zeros, xs))
+    return work
+
+
+def _oracle_step(work):
+    import oracle
+    nbytes = 0
+    for n, K, b, packed, scales, zeros, xs in work:
+        for M in DECODE_MS:
+            oracle.gemm(xs[M], packed, scales, zeros, K, b)
+            nbytes += weight_bytes(n, K, b)
+    return nbytes
+
+
+def cpu_baseline(args):
+    rows = args.cpu_rows
+    work = _oracle_sample(rows)
+    t0 = time.perf_counter()
+    nbytes = _oracle_step(work)
+    dt = time.perf_counter() - t0
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {rows} output rows of each of the 7 block projections, M in {{1,4,16}} "
+                      f"(binary64 scalar C oracle, single thread), {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    rows = args.cpu_rows
+    work = _oracle_sample(rows)
+    for _ in range(args.warmup):
+        _oracle_step(work)
+    t0 = time.perf_counter()
+    nbytes = 0
+    for _ in range(args.steps):
+        nbytes += _oracle_step(work)
+    dt = time.perf_counter() - t0
+    value = nbytes / dt / 1e9
+    sample = (f"first {rows} output rows of each of the 7 Qwen3-8B-block projections, M in {{1,4,16}} "
+              "(binary64 scalar C oracle, single thread)")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "Qwen3-8B-shaped decoder block decode (sampled rows)", "rows_per_layer": rows},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["slq", "reference"], default="slq")
+    ap.add_argument("--repeat", type=int, default=1, help="graph replays per counted step group")
+    ap.add_argument("--headline-only", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=512)
+    args = ap.parse_args()
+    assert args.warmup >= 3 or args.impl == "reference", "at least 3 warm-up steps"
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_slq(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

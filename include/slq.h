@@ -1,0 +1,178 @@
+/*
+ * slq.h -- C ABI of the SLQ weight-format library (libslq.so, sm_100a).
+ *
+ * The library implements the hot path of "Statistically-Lossless
+ * Quantization of Large Language Models" (Helcig, Kurtic, Alistarh): the
+ * layer-wise asymmetric INT-b weight format with group size 128 along K and
+ * a bitwidth b in {2, ..., 8} per layer, and the three operations that run on
+ * it: quantize+pack, the fused dequantize-GEMM, and the EAR/KL fidelity
+ * reduction.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named *_host are host memory; all others are DEVICE memory
+ *     (cudaMalloc or any allocator) owned by the caller.  The library never
+ *     allocates, frees or synchronizes; it only launches kernels on `stream`
+ *     (a cudaStream_t passed as void*, NULL = legacy default stream).
+ *   - Arrays are dense and row-major.  bf16 arrays and packed codes start on
+ *     a 16-byte boundary; the others on their element size (both checked).
+ *     Inputs and outputs must not overlap (checked).
+ *   - bf16 / fp16 data is raw 16-bit IEEE bfloat16 / binary16 bits.
+ *   - Argument errors are reported synchronously, before anything is
+ *     launched.  A failed launch returns SLQ_ERR_CUDA.  Conditions that depend
+ *     on the data are reported asynchronously: kernels OR bits into the
+ *     optional device word *flags (caller zeroes it, reads it after a sync).
+ *   - The only supported device is compute capability 10.0 (B200, sm_100a);
+ *     any other device, or no device, gives SLQ_ERR_UNSUPPORTED_DEVICE.  There
+ *     is no CPU or other-architecture fallback.
+ *   - Calls keep no state between them and may be issued from several host
+ *     threads on different streams.
+ */
+#ifndef SLQ_H
+#define SLQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SLQ_OK = 0,
+  SLQ_ERR_INVALID_ARGUMENT = 1,
+  SLQ_ERR_UNSUPPORTED_DEVICE = 2,
+  SLQ_ERR_CUDA = 3,
+  SLQ_ERR_TIMEOUT = 4
+} slq_status;
+
+typedef enum { SLQ_DTYPE_BF16 = 0, SLQ_DTYPE_F32 = 1 } slq_dtype;
+
+/* Bits OR-ed into *flags by the kernels. */
+enum {
+  SLQ_FLAG_NONFINITE = 1u,      /* a weight was inf or NaN: that group's output is unspecified */
+  SLQ_FLAG_SCALE_OVERFLOW = 2u, /* a group's range exceeded fp16: scale stored as 65504 */
+  SLQ_FLAG_TIMEOUT = 4u         /* a bounded on-chip wait gave up; outputs are unspecified */
+};
+
+/* GEMM kernel choice for slq_gemm_ex. */
+typedef enum {
+  SLQ_GEMM_AUTO = 0,   /* decode kernel for M <= 16, tensor-core tiled kernel above */
+  SLQ_GEMM_DECODE = 1, /* register-dequant mma decode kernel (any M <= 16) */
+  SLQ_GEMM_TILED = 2   /* TMA + tcgen05/TMEM tiled kernel (any M >= 1) */
+} slq_gemm_path;
+
+/* Group size along K, fixed by the format ("asymmetric INT, group size 128",
+ * gist.science summary, Methodology section 3 "The SLQ Pipeline"). */
+#define SLQ_GROUP 128
+
+/* Largest sizes accepted: every row count and K below 2^31, and
+ * N*K, M*K, M*N, T*V below 2^40 elements. */
+
+/* Library version, as 10000*major + 100*minor + patch. */
+int slq_version(void);
+
+/* Human-readable name of a status code (static string). */
+const char *slq_status_string(slq_status status);
+
+/* Number of uint32 words of the packed codes of an [N, K] layer at `bits`
+ * bits: N*K*bits/32 (each 128-code group fills exactly 4*bits words).
+ * Returns 0 for invalid arguments. */
+size_t slq_packed_words(int64_t N, int64_t K, int bits);
+
+/* Which kernel slq_gemm would run for these sizes (SLQ_GEMM_DECODE or
+ * SLQ_GEMM_TILED).  Host-only; launches nothing. */
+slq_gemm_path slq_gemm_select(int64_t M, int64_t N, int64_t K, int bits);
+
+/*
+ * slq_quantize -- round-to-nearest asymmetric INT-`bits` encode of W, group
+ * size 128 along K, packed to the layer's bitwidth.
+ *
+ * Source: the pages fix an asymmetric integer grid, group size 128 and
+ * b in 2..8 per layer (gist.science summary, Methodology section 3 "The SLQ
+ * Pipeline"; GitHub README, "Pipeline" paragraph), round-to-nearest as the
+ * plain encoder (reddit excerpt of the paper's introduction: RTN), and
+ * weights packed to per-layer bitwidths when the model is loaded (GitHub
+ * README, "4. Build and serve a checkpoint").  Per group of 128 weights, in
+ * IEEE binary32: lo = min, hi = max (a constant group is widened to include
+ * 0); s = fp16_rn((hi - lo) / (2^b - 1)) (an all-zero group gets 1.0, a
+ * nonzero step below fp16 range 2^-24, one above it 65504 + flag);
+ * z = clamp(rne(-lo / s), 0, 2^b - 1); q = clamp(rne(w / s) + z, 0, 2^b - 1).
+ *
+ * W_bf16      [N, K] bf16, device, read-only.
+ * N, K        N >= 0 (0 launches nothing), K >= 128 and K % 128 == 0.
+ * bits        2..8.
+ * packed      [N, K*bits/32] uint32, device, written.  Row n is one bit
+ *             stream, least significant bit first (stream bit i is bit i%32
+ *             of word i/32); code k of the row occupies stream bits
+ *             [k*bits, k*bits + bits).
+ * scales_f16  [N, K/128] fp16, device, written.
+ * zeros       [N, K/128] uint8, device, written.
+ * flags       device uint32 or NULL; SLQ_FLAG_NONFINITE / _SCALE_OVERFLOW.
+ * stream      cudaStream_t.
+ */
+slq_status slq_quantize(const void *W_bf16, int64_t N, int64_t K, int bits,
+                        uint32_t *packed, void *scales_f16, uint8_t *zeros,
+                        uint32_t *flags, void *stream);
+
+/*
+ * slq_gemm -- fused dequantize-GEMM Y = X W^T with w[n, k] = s[n, g] *
+ * (q[n, k] - z[n, g]), g = k / 128; bf16 X, fp32 accumulation, bf16 or fp32 Y.
+ *
+ * Source: the weight-only quantized linear layer served with mixed per-layer
+ * bitwidths, to which the pages credit their 1.7-3.7x serving speedup
+ * (gist.science summary, Key Results "Inference Speedup"; GitHub README
+ * intro and "4. Build and serve a checkpoint").
+ *
+ * X_bf16      [M, K] bf16, device.
+ * M, N, K     M >= 0, N >= 0 (either 0 launches nothing), K >= 128, K % 128 == 0.
+ * bits, packed, scales_f16, zeros   as written by slq_quantize.
+ * Y           [M, N] of y_dtype, device, written.  With SLQ_DTYPE_BF16 each
+ *             element is the round-to-nearest-even bf16 of the fp32 value the
+ *             same kernel writes with SLQ_DTYPE_F32 (the reduction order does
+ *             not depend on the output type; no atomics).
+ * flags       device uint32 or NULL; SLQ_FLAG_TIMEOUT.
+ */
+slq_status slq_gemm(const void *X_bf16, int64_t M, int64_t N, int64_t K,
+                    int bits, const uint32_t *packed, const void *scales_f16,
+                    const uint8_t *zeros, void *Y, slq_dtype y_dtype,
+                    uint32_t *flags, void *stream);
+
+/* slq_gemm with an explicit kernel choice (SLQ_GEMM_DECODE needs M <= 16).
+ * Same arguments and results otherwise. */
+slq_status slq_gemm_ex(const void *X_bf16, int64_t M, int64_t N, int64_t K,
+                       int bits, const uint32_t *packed,
+                       const void *scales_f16, const uint8_t *zeros, void *Y,
+                       slq_dtype y_dtype, slq_gemm_path path, uint32_t *flags,
+                       void *stream);
+
+/*
+ * slq_ear_kl -- per-token Expected Acceptance Rate and KL divergence between
+ * the next-token distributions of a reference and a quantized model.
+ *
+ * Source: gist.science summary, Methodology section 2 "Fidelity Metrics"
+ * (EAR = sum over tokens of min(p, q), averaged over positions; KL as the
+ * task-lossless search signal) and the reddit abstract (EAR is the maximum
+ * token-agreement probability under optimal coupling).  The pages restrict
+ * the sum to the top-K tokens in their evaluation; this call sums over the
+ * whole vocabulary (K = V).  With x = a / temperature, y = b / temperature,
+ * p = softmax(x), q = softmax(y):
+ *   ear_tok[t] = sum_v min(p_v, q_v)
+ *   kl_tok[t]  = sum_v p_v (log p_v - log q_v)        (nats)
+ *
+ * logits_p_bf16  [T, V] bf16, device: reference-model logits (p).
+ * logits_q_bf16  [T, V] bf16, device: quantized-model logits (q).
+ * T, V           T >= 0 (0 launches nothing), V >= 1.
+ * temperature    finite, > 0.
+ * ear_tok, kl_tok  [T] fp32, device, written.
+ * ear_mean, kl_mean  device double or NULL: the mean over the T tokens.
+ * flags          device uint32 or NULL; SLQ_FLAG_TIMEOUT.
+ */
+slq_status slq_ear_kl(const void *logits_p_bf16, const void *logits_q_bf16,
+                      int64_t T, int64_t V, float temperature, float *ear_tok,
+                      float *kl_tok, double *ear_mean, double *kl_mean,
+                      uint32_t *flags, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SLQ_H */

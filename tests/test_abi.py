@@ -1,0 +1,117 @@
+"""Host-side checks of the C ABI that need no GPU.
+
+  * libslq.so loads and exports every function include/slq.h declares;
+  * the header carries no torch or CUDA types in its signatures;
+  * argument validation rejects bad calls with SLQ_ERR_INVALID_ARGUMENT
+    before touching CUDA (fake, never-dereferenced pointers are used);
+  * with no CUDA device, a valid call reports SLQ_ERR_UNSUPPORTED_DEVICE;
+  * host helpers (packed_words, gemm_select, status strings).
+"""
+import ctypes
+import re
+import subprocess
+
+import pytest
+import torch
+
+import weight_only_mixed_b200 as slq
+
+L = slq.lib()
+FAKE = 0x7f0000100000  # 16-byte aligned, never dereferenced by validation
+
+
+def test_every_declared_symbol_is_exported():
+    names = slq.declared_symbols()
+    assert {"slq_quantize", "slq_gemm", "slq_ear_kl"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", slq.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (slq_\w+)", out))
+    assert set(names) <= exported
+
+
+def test_header_is_plain_c():
+    with open(slq.HEADER_PATH) as f:
+        text = f.read()
+    code = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    for bad in ("torch", "at::", "cudaStream_t", "#include <cuda", "std::"):
+        assert bad not in code
+    assert 'extern "C"' in code
+
+
+def test_status_strings_and_version():
+    assert slq.status_string(0) == "SLQ_OK"
+    assert "INVALID" in slq.status_string(1)
+    assert slq.version() >= 100
+
+
+def test_packed_words():
+    for b in range(2, 9):
+        assert slq.packed_words(4096, 4096, b) == 4096 * 4096 * b // 32
+        assert slq.packed_words(3, 128, b) == 3 * 4 * b  # 4b words per group
+    assert slq.packed_words(10, 100, 4) == 0
+    assert slq.packed_words(10, 128, 9) == 0
+    assert slq.packed_words(10, 128, 1) == 0
+
+
+def test_gemm_select():
+    assert slq.gemm_select(1, 4096, 4096, 4) == "decode"
+    assert slq.gemm_select(16, 4096, 4096, 4) == "decode"
+    assert slq.gemm_select(17, 4096, 4096, 4) == "tiled"
+    assert slq.gemm_select(4096, 8192, 8192, 2) == "tiled"
+
+
+def _q(N=8, K=256, bits=4, W=FAKE, packed=FAKE + (1 << 24), scales=FAKE + (2 << 24),
+       zeros=FAKE + (3 << 24), flags=None):
+    return L.slq_quantize(W, N, K, bits, packed, scales, zeros, flags, None)
+
+
+def test_quantize_validation():
+    bad = [dict(bits=1), dict(bits=9), dict(K=100), dict(K=0), dict(K=-128), dict(N=-1),
+           dict(W=None), dict(packed=None), dict(scales=None), dict(zeros=None),
+           dict(W=FAKE + 8), dict(packed=FAKE + (1 << 24) + 4), dict(scales=FAKE + (2 << 24) + 1),
+           dict(flags=FAKE + (4 << 24) + 2), dict(N=1 << 31),
+           # output overlapping the input
+           dict(packed=FAKE + 64)]
+    for kw in bad:
+        assert _q(**kw) == slq.SLQ_ERR_INVALID_ARGUMENT, kw
+    assert _q(N=0) == slq.SLQ_OK  # empty: nothing to do, nothing launched
+
+
+def _g(M=4, N=8, K=256, bits=4, X=FAKE, packed=FAKE + (1 << 24), scales=FAKE + (2 << 24),
+       zeros=FAKE + (3 << 24), Y=FAKE + (4 << 24), dtype=0, path=0, flags=None):
+    return L.slq_gemm_ex(X, M, N, K, bits, packed, scales, zeros, Y, dtype, path, flags, None)
+
+
+def test_gemm_validation():
+    bad = [dict(bits=1), dict(bits=9), dict(K=64), dict(K=129), dict(M=-1), dict(N=-1),
+           dict(X=None), dict(Y=None), dict(packed=None), dict(scales=None), dict(zeros=None),
+           dict(X=FAKE + 2), dict(Y=FAKE + (4 << 24) + 8), dict(packed=FAKE + (1 << 24) + 4),
+           dict(dtype=2), dict(path=3), dict(path=1, M=17), dict(Y=FAKE + 16),  # Y overlaps X
+           dict(M=1 << 31)]
+    for kw in bad:
+        assert _g(**kw) == slq.SLQ_ERR_INVALID_ARGUMENT, kw
+    assert _g(M=0) == slq.SLQ_OK and _g(N=0) == slq.SLQ_OK
+
+
+def _e(T=4, V=1000, tau=1.0, a=FAKE, b=FAKE + (1 << 24), ear=FAKE + (2 << 24),
+       kl=FAKE + (3 << 24), em=None, km=None, flags=None):
+    return L.slq_ear_kl(a, b, T, V, tau, ear, kl, em, km, flags, None)
+
+
+def test_ear_kl_validation():
+    bad = [dict(V=0), dict(T=-1), dict(tau=0.0), dict(tau=-1.0), dict(tau=float("inf")),
+           dict(tau=float("nan")), dict(a=None), dict(b=None), dict(ear=None), dict(kl=None),
+           dict(a=FAKE + 2), dict(ear=FAKE + (2 << 24) + 2), dict(em=FAKE + (5 << 24) + 4),
+           dict(ear=FAKE + 8)]  # output overlaps the input
+    for kw in bad:
+        assert _e(**kw) == slq.SLQ_ERR_INVALID_ARGUMENT, kw
+    assert _e(T=0) == slq.SLQ_OK
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device answer")
+def test_valid_calls_without_a_device_are_refused():
+    assert _q() == slq.SLQ_ERR_UNSUPPORTED_DEVICE
+    assert _g() == slq.SLQ_ERR_UNSUPPORTED_DEVICE
+    assert _e() == slq.SLQ_ERR_UNSUPPORTED_DEVICE

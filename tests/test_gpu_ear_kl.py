@@ -1,0 +1,70 @@
+"""GPU parity: slq_ear_kl against the oracle's binary64 EAR/KL, within 1e-5
+absolute per token and for the means."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import weight_only_mixed_b200 as slq
+from gpu_util import Guarded, to_dev_u16, to_host_u16
+
+pytestmark = pytest.mark.gpu
+TOL = 1e-5
+
+
+def _gpu(a_bits, b_bits, tau):
+    T = a_bits.shape[0]
+    ear = Guarded((T,), torch.float32)
+    kl = Guarded((T,), torch.float32)
+    means = Guarded((2,), torch.float64)
+    rc = slq.lib().slq_ear_kl(
+        to_dev_u16(a_bits).data_ptr(), to_dev_u16(b_bits).data_ptr(), T, a_bits.shape[1],
+        float(tau), ear.t.data_ptr(), kl.t.data_ptr(), means.t.data_ptr(),
+        means.t.data_ptr() + 8, None, torch.cuda.current_stream().cuda_stream)
+    assert rc == slq.SLQ_OK
+    torch.cuda.synchronize()
+    assert ear.intact() and kl.intact() and means.intact()
+    m = means.t.cpu().numpy()
+    return ear.t.cpu().numpy(), kl.t.cpu().numpy(), m[0], m[1]
+
+
+@pytest.mark.parametrize("tau", [1.0, 0.7])
+@pytest.mark.parametrize("T,V", [(1, 1), (3, 2), (5, 7), (4, 8), (7, 1000), (3, 3001),
+                                 (2, 65536 + 24), (3, 151936), (2, 151935)])
+def test_matches_oracle(T, V, tau):
+    a, b = synth.logits(T, V, seed=T * 31 + V)
+    e, k, em, km = _gpu(a, b, tau)
+    er, kr = oracle.ear_kl(a, b, tau)
+    assert np.abs(e - er).max() <= TOL
+    assert np.abs(k - kr).max() <= TOL
+    assert abs(em - er.mean()) <= TOL and abs(km - kr.mean()) <= TOL
+
+
+def test_invariants_on_gpu():
+    a, _ = synth.logits(4, 5000, seed=1)
+    e, k, _, _ = _gpu(a, a, 1.0)
+    assert np.abs(e - 1).max() <= TOL and np.abs(k).max() <= TOL
+    la = np.full((2, 64), -1e4)
+    lb = np.full((2, 64), -1e4)
+    la[:, :32] = 0.0
+    lb[:, 32:] = 0.0
+    e, _, _, _ = _gpu(synth.to_bf16_bits(la), synth.to_bf16_bits(lb), 1.0)
+    assert np.abs(e).max() <= TOL
+
+
+@pytest.mark.parametrize("tau", [1.0, 0.7])
+def test_full_size_sampled_tokens(tau):
+    T, V = 4096, 151936
+    a, b = synth.logits_torch(T, V)
+    ear, kl, em, km = slq.ear_kl(a, b, tau)
+    torch.cuda.synchronize()
+    rows = np.sort(np.random.default_rng(int(tau * 10)).choice(T, size=24, replace=False))
+    rows = np.concatenate([[0, T - 1], rows])
+    idx = torch.from_numpy(rows).cuda()
+    er, kr = oracle.ear_kl(to_host_u16(a.index_select(0, idx)), to_host_u16(b.index_select(0, idx)), tau)
+    assert np.abs(ear.index_select(0, idx).cpu().numpy() - er).max() <= TOL
+    assert np.abs(kl.index_select(0, idx).cpu().numpy() - kr).max() <= TOL
+    # the means are plain averages of the per-token values
+    assert abs(em.item() - ear.double().mean().item()) <= 1e-9
+    assert abs(km.item() - kl.double().mean().item()) <= 1e-9

@@ -1,0 +1,132 @@
+"""GPU parity: slq_gemm against the oracle's binary64 GEMM.
+
+Tolerance (the library's contract): on the fp32 output,
+max |y - y_ref| <= 1e-2 * rms(y_ref); on the bf16 output, relative Frobenius
+error <= 4e-3; and the bf16 output equals round-to-nearest-even of the fp32
+output bit for bit (same kernel, same reduction order).  One-hot rows of X
+must reproduce the dequantized weights exactly.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import weight_only_mixed_b200 as slq
+from gpu_util import Guarded, bf16_rn_of_f32, gemm_errors, to_dev_u16, to_host_u16
+
+pytestmark = pytest.mark.gpu
+BITS = [2, 3, 4, 5, 6, 7, 8]
+MAX_TOL = 1e-2
+FROB_TOL = 4e-3
+
+
+def _layer(N, K, bits, seed):
+    w = synth.weights(N, K, seed=seed)
+    packed, scales, zeros, _ = oracle.quantize(w, bits)
+    qw = slq.QuantizedWeight(
+        packed=torch.from_numpy(packed.view(np.int32).copy()).cuda(),
+        scales=to_dev_u16(scales, torch.float16),
+        zeros=torch.from_numpy(zeros.copy()).cuda(), bits=bits, N=N, K=K)
+    return (packed, scales, zeros), qw
+
+
+def _run(x_bits, qw, path):
+    M = x_bits.shape[0]
+    X = to_dev_u16(x_bits)
+    y32 = Guarded((M, qw.N), torch.float32)
+    y16 = Guarded((M, qw.N), torch.bfloat16)
+    slq.gemm(X, qw, out=y32.t, path=path)
+    slq.gemm(X, qw, out=y16.t, path=path)
+    torch.cuda.synchronize()
+    assert y32.intact() and y16.intact()
+    return y32.t.cpu().numpy(), to_host_u16(y16.t)
+
+
+def _check(x_bits, host_layer, qw, path):
+    packed, scales, zeros = host_layer
+    y_ref = oracle.gemm(x_bits, packed, scales, zeros, qw.K, qw.bits)
+    y32, y16 = _run(x_bits, qw, path)
+    mx, _ = gemm_errors(y32, y_ref)
+    _, fro = gemm_errors(synth.bf16_bits_to_f32(y16), y_ref)
+    assert mx <= MAX_TOL, mx
+    assert fro <= FROB_TOL, fro
+    assert np.array_equal(y16, bf16_rn_of_f32(y32))
+    return mx
+
+
+DECODE_SHAPES = [(1, 1, 128), (2, 7, 256), (3, 33, 384), (5, 100, 1152), (8, 1000, 1024),
+                 (9, 64, 2048), (15, 48, 128 * 9), (16, 256, 4096), (4, 300, 128 * 35)]
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("M,N,K", DECODE_SHAPES)
+def test_decode_matches_oracle(bits, M, N, K):
+    host, qw = _layer(N, K, bits, seed=M * 7 + N + K + bits)
+    x = synth.activations(M, K, seed=M + K)
+    _check(x, host, qw, "decode")
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("path", ["decode"])
+def test_one_hot_rows_are_exact(bits, path):
+    N, K = 40, 512
+    host, qw = _layer(N, K, bits, seed=77 + bits)
+    ks = np.array([0, 1, 31, 32, 127, 128, 255, 300, 511, 64, 65, 96, 97, 200, 400, 401])
+    x = np.zeros((len(ks), K))
+    x[np.arange(len(ks)), ks] = 1.0
+    y32, _ = _run(synth.to_bf16_bits(x), qw, path)
+    wdq = oracle.dequantize(*host, K, bits)
+    assert np.array_equal(y32.astype(np.float64), wdq[:, ks].T)
+
+
+def _sampled_layer_check(N, K, bits, Ms, path="auto", n_sample=192):
+    """Full-size layer on the GPU; oracle on all M rows for a sample of
+    output columns (rows of W are independent)."""
+    W = synth.weights_torch(N, K, seed=5000 + N + bits)
+    qw = slq.quantize(W, bits)
+    cols = np.sort(np.random.default_rng(N + K + bits).choice(N, size=min(N, n_sample), replace=False))
+    cols = np.unique(np.concatenate([[0, N - 1], cols]))
+    idx = torch.from_numpy(cols).cuda()
+    from gpu_util import to_host_u32
+    sub = (to_host_u32(qw.packed.index_select(0, idx)), to_host_u16(qw.scales.index_select(0, idx)),
+           qw.zeros.index_select(0, idx).cpu().numpy())
+    for M in Ms:
+        X = synth.activations_torch(M, K, seed=6000 + M)
+        y32 = slq.gemm(X, qw, out_dtype=torch.float32, path=path)
+        y16 = slq.gemm(X, qw, out_dtype=torch.bfloat16, path=path)
+        torch.cuda.synchronize()
+        y_ref = oracle.gemm(to_host_u16(X), *sub, K, bits)
+        g32 = y32.index_select(1, idx).cpu().numpy()
+        g16 = to_host_u16(y16.index_select(1, idx))
+        mx, _ = gemm_errors(g32, y_ref)
+        _, fro = gemm_errors(synth.bf16_bits_to_f32(g16), y_ref)
+        assert mx <= MAX_TOL and fro <= FROB_TOL, (M, mx, fro)
+        assert np.array_equal(g16, bf16_rn_of_f32(g32))
+
+
+def test_config0_single_linear_full():
+    host, qw = _layer(1024, 1024, 4, seed=synth.SEED_WEIGHTS)
+    x = synth.activations(8, 1024, seed=synth.SEED_X)
+    _check(x, host, qw, "auto")
+
+
+QWEN3_8B = [(4096, 4096, 5), (1024, 4096, 8), (1024, 4096, 8), (4096, 4096, 5),
+            (12288, 4096, 4), (12288, 4096, 4), (4096, 12288, 4)]
+LLAMA_70B = [(8192, 8192, 7), (1024, 8192, 8), (1024, 8192, 8), (8192, 8192, 7),
+             (28672, 8192, 6), (28672, 8192, 6), (8192, 28672, 6)]
+
+
+@pytest.mark.parametrize("N,K,bits", sorted(set(QWEN3_8B)))
+def test_qwen3_8b_block_decode(N, K, bits):
+    _sampled_layer_check(N, K, bits, Ms=[1, 4, 16])
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_sweep_8192_decode(bits):
+    _sampled_layer_check(8192, 8192, bits, Ms=[1, 16], n_sample=96)
+
+
+@pytest.mark.parametrize("N,K,bits", sorted(set(LLAMA_70B)))
+def test_llama_70b_block_decode(N, K, bits):
+    _sampled_layer_check(N, K, bits, Ms=[1, 16], n_sample=64)

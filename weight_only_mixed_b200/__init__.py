@@ -1,0 +1,194 @@
+"""Python binding of libslq.so, the sm_100a library for the SLQ weight format.
+
+This module only marshals arguments: it allocates outputs with PyTorch,
+passes raw device pointers and the current CUDA stream through the C ABI
+declared in ``include/slq.h``, and turns status codes into exceptions.  Every
+step of quantize, dequantize-GEMM and EAR/KL runs in the library's CUDA
+kernels; there is no CPU path and no fallback.  If the library has not been
+built, importing this package fails.
+
+Format (pages on "Statistically-Lossless Quantization of Large Language
+Models"): asymmetric INT-b, b in 2..8 per layer, group size 128 along K,
+fp16 scale and uint8 zero point per group, codes packed LSB-first into one
+bit stream per row (a 128-code group fills exactly 4b uint32 words).
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+import re
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libslq.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "slq.h")
+
+GROUP = 128
+
+SLQ_OK = 0
+SLQ_ERR_INVALID_ARGUMENT = 1
+SLQ_ERR_UNSUPPORTED_DEVICE = 2
+SLQ_ERR_CUDA = 3
+SLQ_ERR_TIMEOUT = 4
+
+SLQ_DTYPE_BF16 = 0
+SLQ_DTYPE_F32 = 1
+
+SLQ_FLAG_NONFINITE = 1
+SLQ_FLAG_SCALE_OVERFLOW = 2
+SLQ_FLAG_TIMEOUT = 4
+
+SLQ_GEMM_AUTO = 0
+SLQ_GEMM_DECODE = 1
+SLQ_GEMM_TILED = 2
+
+_PATHS = {"auto": SLQ_GEMM_AUTO, "decode": SLQ_GEMM_DECODE, "tiled": SLQ_GEMM_TILED}
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m weight_only_mixed_b200.build` "
+        "(nvcc, sm_100a).  There is no fallback implementation.")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I = ctypes.c_int
+
+_lib.slq_version.argtypes = []
+_lib.slq_version.restype = _I
+_lib.slq_status_string.argtypes = [_I]
+_lib.slq_status_string.restype = ctypes.c_char_p
+_lib.slq_packed_words.argtypes = [_I64, _I64, _I]
+_lib.slq_packed_words.restype = ctypes.c_size_t
+_lib.slq_gemm_select.argtypes = [_I64, _I64, _I64, _I]
+_lib.slq_gemm_select.restype = _I
+_lib.slq_quantize.argtypes = [_P, _I64, _I64, _I, _P, _P, _P, _P, _P]
+_lib.slq_quantize.restype = _I
+_lib.slq_gemm.argtypes = [_P, _I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _P, _P]
+_lib.slq_gemm.restype = _I
+_lib.slq_gemm_ex.argtypes = [_P, _I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _I, _P, _P]
+_lib.slq_gemm_ex.restype = _I
+_lib.slq_ear_kl.argtypes = [_P, _P, _I64, _I64, ctypes.c_float, _P, _P, _P, _P, _P, _P]
+_lib.slq_ear_kl.restype = _I
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (for callers that pass raw pointers)."""
+    return _lib
+
+
+def declared_symbols() -> list[str]:
+    """Names of the functions include/slq.h declares."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(slq_[a-z0-9_]+)\s*\(", text)))
+
+
+class SLQError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}")
+
+
+def status_string(status: int) -> str:
+    return _lib.slq_status_string(status).decode()
+
+
+def version() -> int:
+    return _lib.slq_version()
+
+
+def packed_words(N: int, K: int, bits: int) -> int:
+    return int(_lib.slq_packed_words(N, K, bits))
+
+
+def gemm_select(M: int, N: int, K: int, bits: int) -> str:
+    return {SLQ_GEMM_DECODE: "decode", SLQ_GEMM_TILED: "tiled"}[_lib.slq_gemm_select(M, N, K, bits)]
+
+
+def _check(status: int, what: str):
+    if status != SLQ_OK:
+        raise SLQError(status, what)
+
+
+def _stream_ptr(stream=None) -> int:
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else int(t.data_ptr())
+
+
+@dataclasses.dataclass
+class QuantizedWeight:
+    """Packed layer: codes [N, K*b/32] (int32 storage of uint32 words),
+    scales [N, K/128] fp16, zeros [N, K/128] uint8."""
+    packed: "object"
+    scales: "object"
+    zeros: "object"
+    bits: int
+    N: int
+    K: int
+
+    @property
+    def nbytes(self) -> int:
+        """Bytes the GEMM streams: codes + scales + zeros."""
+        return self.N * self.K * self.bits // 8 + self.N * (self.K // GROUP) * 3
+
+
+def empty_quantized(N: int, K: int, bits: int, device="cuda") -> QuantizedWeight:
+    import torch
+    return QuantizedWeight(
+        packed=torch.empty((N, K * bits // 32), dtype=torch.int32, device=device),
+        scales=torch.empty((N, K // GROUP), dtype=torch.float16, device=device),
+        zeros=torch.empty((N, K // GROUP), dtype=torch.uint8, device=device),
+        bits=bits, N=N, K=K)
+
+
+def quantize(W, bits: int, out: QuantizedWeight | None = None, flags=None, stream=None) -> QuantizedWeight:
+    """Quantize a [N, K] bf16 CUDA tensor to the `bits`-bit packed format."""
+    import torch
+    assert W.dtype == torch.bfloat16 and W.is_cuda and W.is_contiguous() and W.dim() == 2
+    N, K = W.shape
+    q = out if out is not None else empty_quantized(N, K, bits, W.device)
+    _check(_lib.slq_quantize(_ptr(W), N, K, bits, _ptr(q.packed), _ptr(q.scales), _ptr(q.zeros),
+                             _ptr(flags), _stream_ptr(stream)), "slq_quantize")
+    return q
+
+
+def gemm(X, qw: QuantizedWeight, out_dtype=None, path: str = "auto", out=None, flags=None,
+         stream=None):
+    """Y = X W^T for bf16 X [M, K] and a packed layer; Y is bf16 or fp32 [M, N]."""
+    import torch
+    out_dtype = out_dtype or torch.bfloat16
+    assert X.dtype == torch.bfloat16 and X.is_cuda and X.is_contiguous() and X.dim() == 2
+    M, K = X.shape
+    assert K == qw.K
+    y = out if out is not None else torch.empty((M, qw.N), dtype=out_dtype, device=X.device)
+    dt = SLQ_DTYPE_F32 if y.dtype == torch.float32 else SLQ_DTYPE_BF16
+    _check(_lib.slq_gemm_ex(_ptr(X), M, qw.N, K, qw.bits, _ptr(qw.packed), _ptr(qw.scales),
+                            _ptr(qw.zeros), _ptr(y), dt, _PATHS[path], _ptr(flags),
+                            _stream_ptr(stream)), "slq_gemm")
+    return y
+
+
+def ear_kl(a, b, temperature: float = 1.0, means: bool = True, flags=None, stream=None):
+    """Per-token EAR and KL(p || q) of two [T, V] bf16 logit tensors.
+
+    Returns (ear_tok, kl_tok, ear_mean, kl_mean); the means are 0-d float64
+    tensors on the device (None when means=False)."""
+    import torch
+    assert a.dtype == torch.bfloat16 and b.dtype == torch.bfloat16 and a.shape == b.shape
+    assert a.is_contiguous() and b.is_contiguous() and a.dim() == 2
+    T, V = a.shape
+    ear = torch.empty(T, dtype=torch.float32, device=a.device)
+    kl = torch.empty(T, dtype=torch.float32, device=a.device)
+    em = torch.empty((), dtype=torch.float64, device=a.device) if means else None
+    km = torch.empty((), dtype=torch.float64, device=a.device) if means else None
+    _check(_lib.slq_ear_kl(_ptr(a), _ptr(b), T, V, float(temperature), _ptr(ear), _ptr(kl),
+                           _ptr(em), _ptr(km), _ptr(flags), _stream_ptr(stream)), "slq_ear_kl")
+    return ear, kl, em, km

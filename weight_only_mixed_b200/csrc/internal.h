@@ -1,0 +1,39 @@
+// internal.h -- launchers shared between the C-ABI front end (slq_api.cu) and
+// the kernel translation units.  Not part of the public ABI (see include/slq.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace slq {
+
+constexpr int kGroup = 128;  // group size along K fixed by the format
+
+// Flag bits (same values as SLQ_FLAG_* in slq.h).
+constexpr uint32_t kFlagNonfinite = 1u;
+constexpr uint32_t kFlagScaleOverflow = 2u;
+constexpr uint32_t kFlagTimeout = 4u;
+
+cudaError_t launch_quantize(const uint16_t* W, int64_t N, int64_t K, int bits,
+                            uint32_t* packed, uint16_t* scales, uint8_t* zeros,
+                            uint32_t* flags, cudaStream_t stream);
+
+// Decode GEMV/skinny GEMM for M <= 16 (register dequant + mma.sync).
+cudaError_t launch_gemm_decode(const uint16_t* X, int64_t M, int64_t N, int64_t K,
+                               int bits, const uint32_t* packed,
+                               const uint16_t* scales, const uint8_t* zeros,
+                               void* Y, bool y_f32, cudaStream_t stream);
+
+// Tiled GEMM (TMA + dequant-to-smem + tcgen05.mma with TMEM accumulators).
+cudaError_t launch_gemm_tiled(const uint16_t* X, int64_t M, int64_t N, int64_t K,
+                              int bits, const uint32_t* packed,
+                              const uint16_t* scales, const uint8_t* zeros,
+                              void* Y, bool y_f32, uint32_t* flags,
+                              cudaStream_t stream);
+
+cudaError_t launch_ear_kl(const uint16_t* a, const uint16_t* b, int64_t T, int64_t V,
+                          float temperature, float* ear_tok, float* kl_tok,
+                          double* ear_mean, double* kl_mean, uint32_t* flags,
+                          cudaStream_t stream);
+
+}  // namespace slq
