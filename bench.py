@@ -352,7 +352,7 @@ def run_slq(args, rank, world, local_rank):
             },
             "roofline": {
                 "bound": "hbm",
-                "kernel": "gemm_decode_kernel (register dequant + mma.m16n8k16, M<=16)",
+                "kernel": "gemm_tiled_kernel<b, BN=16> (TMA + dequant to smem + tcgen05.mma/TMEM, split-K cluster; M<=16)",
                 "achieved": round(achieved, 1),
                 "peak": hbm_peak,
                 "unit": "GB/s",
@@ -432,6 +432,37 @@ def other_rows(args, slq, synth, torch, dev, stream, hbm_peak, tc_peak, rank):
                                    "us": round(ms * 1e3, 2)}
         del qws
     rows["decode_sweep_8192"] = sweep
+
+    # Tiled (prefill) GEMM: N = K = 8192 at M in {1024, 4096}, and the
+    # Llama-3.3-70B-shaped block at M = 2048; TFLOP/s on 2*M*N*K.
+    pre = {}
+    for (name, N, K, b, M) in [("sweep8192_b2", 8192, 8192, 2, 1024), ("sweep8192_b4", 8192, 8192, 4, 1024),
+                               ("sweep8192_b8", 8192, 8192, 8, 1024), ("sweep8192_b2", 8192, 8192, 2, 4096),
+                               ("sweep8192_b4", 8192, 8192, 4, 4096), ("sweep8192_b8", 8192, 8192, 8, 4096)]:
+        qw = slq.quantize(synth.weights_torch(N, K, seed=900 + b, device=dev), b)
+        Xp = synth.activations_torch(M, K, seed=901, device=dev)
+        Yp = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ms = time_ms(torch, stream, lambda: slq.gemm(Xp, qw, out=Yp, stream=stream), 10)
+        tf = 2 * M * N * K / (ms * 1e-3) / 1e12
+        pre[f"{name}_M{M}"] = {"TFLOPs": round(tf, 1), "frac_tensor": round(tf / tc_peak, 3), "us": round(ms * 1e3, 1)}
+        del qw, Xp, Yp
+    llama = [(8192, 8192, 7), (1024, 8192, 8), (1024, 8192, 8), (8192, 8192, 7), (28672, 8192, 6),
+             (28672, 8192, 6), (8192, 28672, 6)]
+    M = 2048
+    qws = [slq.quantize(synth.weights_torch(N, K, seed=950 + i, device=dev), b) for i, (N, K, b) in enumerate(llama)]
+    Xs = [synth.activations_torch(M, K, seed=960 + i, device=dev) for i, (N, K, b) in enumerate(llama)]
+    Ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for (N, K, b) in llama]
+
+    def block():
+        for x, q, y in zip(Xs, qws, Ys):
+            slq.gemm(x, q, out=y, stream=stream)
+
+    ms = time_ms(torch, stream, block, 5)
+    flops = sum(2 * M * N * K for (N, K, b) in llama)
+    tf = flops / (ms * 1e-3) / 1e12
+    pre["llama70b_block_M2048"] = {"TFLOPs": round(tf, 1), "frac_tensor": round(tf / tc_peak, 3), "us": round(ms * 1e3, 1)}
+    del qws, Xs, Ys
+    rows["tiled_prefill"] = pre
 
     # EAR / KL over [4096 x 151936] bf16 logits, tau 1.0 and 0.7.
     T, V = 4096, 151936

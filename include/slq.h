@@ -54,11 +54,14 @@ enum {
   SLQ_FLAG_TIMEOUT = 4u         /* a bounded on-chip wait gave up; outputs are unspecified */
 };
 
-/* GEMM kernel choice for slq_gemm_ex. */
+/* GEMM kernel configuration for slq_gemm_ex.  Every configuration runs the
+ * same sm_100a kernel: TMA-staged packed weights, dequantized to exact bf16
+ * (q - z) in shared memory, tcgen05.mma into TMEM per 128-wide group, and the
+ * fp16 group scale applied to the fp32 group product. */
 typedef enum {
-  SLQ_GEMM_AUTO = 0,   /* decode kernel for M <= 16, tensor-core tiled kernel above */
-  SLQ_GEMM_DECODE = 1, /* register-dequant mma decode kernel (any M <= 16) */
-  SLQ_GEMM_TILED = 2   /* TMA + tcgen05/TMEM tiled kernel (any M >= 1) */
+  SLQ_GEMM_AUTO = 0,   /* DECODE for M <= 16, TILED above */
+  SLQ_GEMM_DECODE = 1, /* 128 x 16 output tiles, K split over a thread-block cluster (M <= 16) */
+  SLQ_GEMM_TILED = 2   /* 128 x {64, 128, 256} output tiles sized to M (any M >= 1) */
 } slq_gemm_path;
 
 /* Group size along K, fixed by the format ("asymmetric INT, group size 128",

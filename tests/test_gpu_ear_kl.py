@@ -18,8 +18,9 @@ def _gpu(a_bits, b_bits, tau):
     ear = Guarded((T,), torch.float32)
     kl = Guarded((T,), torch.float32)
     means = Guarded((2,), torch.float64)
+    A, Bq = to_dev_u16(a_bits), to_dev_u16(b_bits)  # keep both alive during the call
     rc = slq.lib().slq_ear_kl(
-        to_dev_u16(a_bits).data_ptr(), to_dev_u16(b_bits).data_ptr(), T, a_bits.shape[1],
+        A.data_ptr(), Bq.data_ptr(), T, a_bits.shape[1],
         float(tau), ear.t.data_ptr(), kl.t.data_ptr(), means.t.data_ptr(),
         means.t.data_ptr() + 8, None, torch.cuda.current_stream().cuda_stream)
     assert rc == slq.SLQ_OK

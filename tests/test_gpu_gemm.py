@@ -68,7 +68,7 @@ def test_decode_matches_oracle(bits, M, N, K):
 
 
 @pytest.mark.parametrize("bits", BITS)
-@pytest.mark.parametrize("path", ["decode"])
+@pytest.mark.parametrize("path", ["decode", "tiled"])
 def test_one_hot_rows_are_exact(bits, path):
     N, K = 40, 512
     host, qw = _layer(N, K, bits, seed=77 + bits)
@@ -130,3 +130,55 @@ def test_sweep_8192_decode(bits):
 @pytest.mark.parametrize("N,K,bits", sorted(set(LLAMA_70B)))
 def test_llama_70b_block_decode(N, K, bits):
     _sampled_layer_check(N, K, bits, Ms=[1, 16], n_sample=64)
+
+
+# ---------------------------------------------------------------------------
+# Tiled tensor-core path (TMA + dequant-to-smem + tcgen05.mma, TMEM accumulators)
+# ---------------------------------------------------------------------------
+TILED_SHAPES = [(17, 1, 128), (40, 130, 256), (64, 128, 384), (65, 257, 1024), (128, 100, 640),
+                (129, 384, 512), (200, 64, 1152), (256, 256, 2048), (300, 200, 768), (1, 50, 256),
+                (16, 129, 128 * 5)]
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("M,N,K", TILED_SHAPES)
+def test_tiled_matches_oracle(bits, M, N, K):
+    host, qw = _layer(N, K, bits, seed=M * 13 + N + K + bits)
+    x = synth.activations(M, K, seed=M + K + 1)
+    _check(x, host, qw, "tiled")
+
+
+def _sampled_prefill_check(N, K, bits, Ms, n_rows=48, n_cols=160, path="auto"):
+    W = synth.weights_torch(N, K, seed=7000 + N + bits)
+    qw = slq.quantize(W, bits)
+    del W
+    from gpu_util import to_host_u32
+    rng = np.random.default_rng(N + K + bits)
+    cols = np.unique(np.concatenate([[0, N - 1], rng.choice(N, size=min(N, n_cols), replace=False)]))
+    cidx = torch.from_numpy(cols).cuda()
+    sub = (to_host_u32(qw.packed.index_select(0, cidx)), to_host_u16(qw.scales.index_select(0, cidx)),
+           qw.zeros.index_select(0, cidx).cpu().numpy())
+    for M in Ms:
+        X = synth.activations_torch(M, K, seed=8000 + M)
+        y32 = slq.gemm(X, qw, out_dtype=torch.float32, path=path)
+        y16 = slq.gemm(X, qw, out_dtype=torch.bfloat16, path=path)
+        torch.cuda.synchronize()
+        rows = np.unique(np.concatenate([[0, M - 1], rng.choice(M, size=min(M, n_rows), replace=False)]))
+        ridx = torch.from_numpy(rows).cuda()
+        y_ref = oracle.gemm(to_host_u16(X.index_select(0, ridx)), *sub, K, bits)
+        g32 = y32.index_select(0, ridx).index_select(1, cidx).cpu().numpy()
+        g16 = to_host_u16(y16.index_select(0, ridx).index_select(1, cidx))
+        mx, _ = gemm_errors(g32, y_ref)
+        _, fro = gemm_errors(synth.bf16_bits_to_f32(g16), y_ref)
+        assert mx <= MAX_TOL and fro <= FROB_TOL, (M, mx, fro)
+        assert np.array_equal(g16, bf16_rn_of_f32(g32))
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_sweep_8192_prefill(bits):
+    _sampled_prefill_check(8192, 8192, bits, Ms=[64, 256, 1024, 4096])
+
+
+@pytest.mark.parametrize("N,K,bits", sorted(set(LLAMA_70B)))
+def test_llama_70b_block_prefill(N, K, bits):
+    _sampled_prefill_check(N, K, bits, Ms=[64, 2048])

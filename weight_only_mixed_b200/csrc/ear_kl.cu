@@ -15,10 +15,13 @@
 // log-domain form needs no per-element logarithm and has no 0 * log 0 case.
 // Differences of two bf16 logits are exact in fp32, so every exponent argument
 // is one rounding away from exact.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
 #include "internal.h"
 #include "ptx.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace slq {
 namespace {
@@ -211,6 +214,266 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Cluster kernel (V % 8 == 0): one HBM pass.  A cluster of 8 CTAs owns one
+// token row at a time; CTA r keeps slice r of both logit rows in shared memory
+// (double-buffered 1-D bulk copies, the next row lands while this one is
+// processed).  Per row: local max, local sums -> statistics exchanged through
+// distributed shared memory and merged in rank order -> the EAR sum from the
+// resident slice.  The EAR partials of row i are added up by rank 0 after the
+// exchange of row i+1, so each row costs a single cluster barrier.
+// ---------------------------------------------------------------------------
+constexpr int kClusterCtas = 8;
+constexpr int kClusterThreads = 512;
+
+struct SliceStat {
+  float ma, sa, w, mb, sb;
+};
+
+template <int kThreads>
+__device__ float2 block_max2(float x, float y, float* red) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    x = fmaxf(x, __shfl_xor_sync(kFull, x, off));
+    y = fmaxf(y, __shfl_xor_sync(kFull, y, off));
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    red[2 * warp] = x;
+    red[2 * warp + 1] = y;
+  }
+  __syncthreads();
+  float rx = red[0], ry = red[1];
+  for (int w = 1; w < kThreads / 32; ++w) {
+    rx = fmaxf(rx, red[2 * w]);
+    ry = fmaxf(ry, red[2 * w + 1]);
+  }
+  __syncthreads();
+  return make_float2(rx, ry);
+}
+
+// Sum of three values over the block, fixed order; valid in every thread.
+template <int kThreads>
+__device__ float3 block_sum3(float x, float y, float z, float* red) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    x += __shfl_xor_sync(kFull, x, off);
+    y += __shfl_xor_sync(kFull, y, off);
+    z += __shfl_xor_sync(kFull, z, off);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    red[3 * warp] = x;
+    red[3 * warp + 1] = y;
+    red[3 * warp + 2] = z;
+  }
+  __syncthreads();
+  float rx = 0.0f, ry = 0.0f, rz = 0.0f;
+  for (int w = 0; w < kThreads / 32; ++w) {
+    rx += red[3 * w];
+    ry += red[3 * w + 1];
+    rz += red[3 * w + 2];
+  }
+  __syncthreads();
+  return make_float3(rx, ry, rz);
+}
+
+__global__ void __launch_bounds__(kClusterThreads, 1)
+    ear_kl_cluster_kernel(const uint16_t* __restrict__ A, const uint16_t* __restrict__ Bq,
+                          int64_t T, int64_t V, int units_per_cta, float c, float inv_temp,
+                          float* __restrict__ ear_tok, float* __restrict__ kl_tok,
+                          uint32_t* __restrict__ flags) {
+  constexpr uint64_t kWaitLimitNs = 2000000000ull;
+  extern __shared__ __align__(128) uint8_t smem[];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int64_t cluster_id = blockIdx.x / kClusterCtas;
+  const int64_t nclusters = gridDim.x / kClusterCtas;
+
+  const int64_t v8 = V / 8;
+  const int64_t r0 = static_cast<int64_t>(rank) * units_per_cta;
+  const int64_t u0 = r0 < v8 ? r0 : v8;
+  const int64_t u1 = (u0 + units_per_cta) < v8 ? (u0 + units_per_cta) : v8;
+  const int nu = static_cast<int>(u1 - u0);  // 16-byte units of this CTA's slice
+  const size_t slice_bytes = static_cast<size_t>(units_per_cta) * 16;
+
+  // [buf][tensor][slice] | barriers | stats[2] | ear[2] | merged | reduction scratch
+  uint8_t* data = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(data + 4 * slice_bytes);
+  SliceStat* stats = reinterpret_cast<SliceStat*>(full + 2);
+  float* ear_part = reinterpret_cast<float*>(stats + 2);
+  SliceStat* merged = reinterpret_cast<SliceStat*>(ear_part + 2);
+  float* red = reinterpret_cast<float*>(merged + 1);
+  __shared__ int aborted;
+
+  const int64_t nrows = (T > cluster_id) ? (T - cluster_id + nclusters - 1) / nclusters : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
+    aborted = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  cluster.sync();  // every CTA of the cluster is running before any remote access
+
+  auto issue = [&](int64_t i) {
+    const int buf = static_cast<int>(i & 1);
+    const int64_t t = cluster_id + i * nclusters;
+    uint8_t* da = data + (2 * buf) * slice_bytes;
+    uint8_t* db = data + (2 * buf + 1) * slice_bytes;
+    const uint32_t bytes = static_cast<uint32_t>(nu) * 16;
+    mbar_arrive_expect_tx(&full[buf], 2 * bytes);
+    if (bytes) {
+      bulk_load(da, A + t * V + u0 * 8, bytes, &full[buf]);
+      bulk_load(db, Bq + t * V + u0 * 8, bytes, &full[buf]);
+    }
+  };
+  int64_t issued = 0;
+  if (threadIdx.x == 0) {
+    for (; issued < 2 && issued < nrows; ++issued) issue(issued);
+  }
+
+  for (int64_t i = 0; i < nrows; ++i) {
+    const int buf = static_cast<int>(i & 1);
+    const int64_t t = cluster_id + i * nclusters;
+    if (!aborted) {
+      if (!mbar_wait_bounded(&full[buf], static_cast<uint32_t>((i >> 1) & 1), kWaitLimitNs)) {
+        aborted = 1;
+        if (flags) atomicOr(flags, kFlagTimeout);
+      }
+    }
+    __syncthreads();
+    const bool live = !aborted;
+    const uint4* sa4 = reinterpret_cast<const uint4*>(data + (2 * buf) * slice_bytes);
+    const uint4* sb4 = reinterpret_cast<const uint4*>(data + (2 * buf + 1) * slice_bytes);
+
+    // Local maxima of the raw logits (the temperature scale is monotone).
+    float mxa = -INFINITY, mxb = -INFINITY;
+    if (live) {
+      for (int k = threadIdx.x; k < nu; k += kClusterThreads) {
+        const uint4 va = sa4[k], vb = sb4[k];
+        const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
+        const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          mxa = fmaxf(mxa, fmaxf(bf16_lo(wa[q]), bf16_hi(wa[q])));
+          mxb = fmaxf(mxb, fmaxf(bf16_lo(wb[q]), bf16_hi(wb[q])));
+        }
+      }
+    }
+    const float2 mx = block_max2<kClusterThreads>(mxa, mxb, red);
+    // Local sums around the local maxima.
+    float s_a = 0.0f, s_b = 0.0f, w_ab = 0.0f;
+    if (live && nu > 0) {
+      for (int k = threadIdx.x; k < nu; k += kClusterThreads) {
+        const uint4 va = sa4[k], vb = sb4[k];
+        const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
+        const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float a0 = bf16_lo(wa[q]), a1 = bf16_hi(wa[q]);
+          const float b0 = bf16_lo(wb[q]), b1 = bf16_hi(wb[q]);
+          const float e0 = ex2((a0 - mx.x) * c), e1 = ex2((a1 - mx.x) * c);
+          s_a += e0 + e1;
+          w_ab = fmaf(e0, a0 - b0, fmaf(e1, a1 - b1, w_ab));
+          s_b += ex2((b0 - mx.y) * c) + ex2((b1 - mx.y) * c);
+        }
+      }
+    }
+    const float3 sums = block_sum3<kClusterThreads>(s_a, s_b, w_ab, red);
+    if (threadIdx.x == 0) stats[buf] = SliceStat{mx.x, sums.x, sums.z, mx.y, sums.y};
+
+    cluster.sync();  // statistics of row i (and EAR partials of row i-1) are visible
+
+    if (threadIdx.x < 32) {
+      // Merge the 8 slices in rank order (lane 0 does the fixed-order sums).
+      SliceStat r = {-INFINITY, 0.0f, 0.0f, -INFINITY, 0.0f};
+      if (threadIdx.x < kClusterCtas) r = cluster.map_shared_rank(stats, static_cast<int>(threadIdx.x))[buf];
+      float prev_ear = 0.0f;
+      if (rank == 0 && i > 0 && threadIdx.x < kClusterCtas)
+        prev_ear = cluster.map_shared_rank(ear_part, static_cast<int>(threadIdx.x))[buf ^ 1];
+      SliceStat all[kClusterCtas];
+      float pe[kClusterCtas];
+#pragma unroll
+      for (int j = 0; j < kClusterCtas; ++j) {
+        all[j].ma = __shfl_sync(kFull, r.ma, j);
+        all[j].sa = __shfl_sync(kFull, r.sa, j);
+        all[j].w = __shfl_sync(kFull, r.w, j);
+        all[j].mb = __shfl_sync(kFull, r.mb, j);
+        all[j].sb = __shfl_sync(kFull, r.sb, j);
+        pe[j] = __shfl_sync(kFull, prev_ear, j);
+      }
+      if (threadIdx.x == 0) {
+        float Ma = -INFINITY, Mb = -INFINITY;
+        for (int j = 0; j < kClusterCtas; ++j) {
+          Ma = fmaxf(Ma, all[j].ma);
+          Mb = fmaxf(Mb, all[j].mb);
+        }
+        float Sa = 0.0f, Sb = 0.0f, W = 0.0f;
+        for (int j = 0; j < kClusterCtas; ++j) {
+          if (all[j].ma != -INFINITY) {
+            const float f = ex2((all[j].ma - Ma) * c);
+            Sa = fmaf(all[j].sa, f, Sa);
+            W = fmaf(all[j].w, f, W);
+          }
+          if (all[j].mb != -INFINITY) Sb = fmaf(all[j].sb, ex2((all[j].mb - Mb) * c), Sb);
+        }
+        *merged = SliceStat{Ma, Sa, W, Mb, Sb};
+        if (rank == 0) {
+          constexpr float kLn2 = 0.693147180559945309f;
+          const float la = lg2(Sa), lb = lg2(Sb);
+          if (live) kl_tok[t] = (W / Sa) * inv_temp - ((Ma - Mb) * inv_temp + (la - lb) * kLn2);
+          if (i > 0) {
+            float e = 0.0f;
+            for (int j = 0; j < kClusterCtas; ++j) e += pe[j];
+            ear_tok[t - nclusters] = e;
+          }
+        }
+      }
+    }
+    __syncthreads();
+    const SliceStat g = *merged;
+    const float la = lg2(g.sa), lb = lg2(g.sb);
+
+    // EAR terms of the resident slice: sum 2^min(log2 p, log2 q).
+    float e_acc[2] = {0.0f, 0.0f};
+    if (live) {
+      for (int k = threadIdx.x; k < nu; k += kClusterThreads) {
+        const uint4 va = sa4[k], vb = sb4[k];
+        const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
+        const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          e_acc[q & 1] += ex2(fminf((bf16_lo(wa[q]) - g.ma) * c - la, (bf16_lo(wb[q]) - g.mb) * c - lb));
+          e_acc[q & 1] += ex2(fminf((bf16_hi(wa[q]) - g.ma) * c - la, (bf16_hi(wb[q]) - g.mb) * c - lb));
+        }
+      }
+    }
+    const float3 es = block_sum3<kClusterThreads>(e_acc[0] + e_acc[1], 0.0f, 0.0f, red);
+    if (threadIdx.x == 0) ear_part[buf] = es.x;
+    // block_sum3 ended with __syncthreads: every read of this buffer is done.
+    if (threadIdx.x == 0 && !aborted && issued < nrows && issued == i + 2) {
+      fence_proxy_async_smem();
+      issue(issued);
+      ++issued;
+    }
+  }
+  cluster.sync();  // EAR partials of the last row are visible
+  if (rank == 0 && threadIdx.x == 0 && nrows > 0) {
+    const int buf = static_cast<int>((nrows - 1) & 1);
+    float e = 0.0f;
+    for (int j = 0; j < kClusterCtas; ++j) e += cluster.map_shared_rank(ear_part, j)[buf];
+    ear_tok[cluster_id + (nrows - 1) * nclusters] = e;
+  }
+  // Copies issued but never consumed (only after a timeout) must land first.
+  if (threadIdx.x == 0 && aborted) {
+    for (int64_t i = (issued > 2 ? issued - 2 : 0); i < issued; ++i)
+      mbar_wait_bounded(&full[i & 1], static_cast<uint32_t>((i >> 1) & 1), kWaitLimitNs);
+  }
+  cluster.sync();  // keep shared memory alive until rank 0 has read it
+}
+
 // Means over tokens in binary64, one block, fixed summation order.
 __global__ void __launch_bounds__(1024)
     token_mean_kernel(const float* __restrict__ ear_tok, const float* __restrict__ kl_tok,
@@ -237,27 +500,68 @@ __global__ void __launch_bounds__(1024)
   }
 }
 
+constexpr size_t kClusterSmemExtra = 16 + 2 * sizeof(SliceStat) + 8 + sizeof(SliceStat) +
+                                     (3 * (kClusterThreads / 32) + 2) * sizeof(float) + 64;
+
 }  // namespace
 
 cudaError_t launch_ear_kl(const uint16_t* a, const uint16_t* b, int64_t T, int64_t V,
                           float temperature, float* ear_tok, float* kl_tok, double* ear_mean,
                           double* kl_mean, uint32_t* flags, cudaStream_t stream) {
-  (void)flags;
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const float inv_temp = 1.0f / temperature;
   const float c = 1.4426950408889634f * inv_temp;
-  constexpr int kThreads = 1024;
-  int64_t blocks = T < static_cast<int64_t>(sms) * 2 ? T : static_cast<int64_t>(sms) * 2;
-  if (V % 8 == 0)
-    ear_kl_rows_kernel<kThreads, true><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
-        a, b, T, V, c, inv_temp, ear_tok, kl_tok);
-  else
-    ear_kl_rows_kernel<kThreads, false><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
-        a, b, T, V, c, inv_temp, ear_tok, kl_tok);
-  cudaError_t err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
+  cudaError_t err = cudaSuccess;
+
+  // Single-pass cluster kernel when rows are 16-byte aligned and a slice pair
+  // (double-buffered) fits in shared memory; the row kernel otherwise.
+  const int64_t v8 = V / 8;
+  const int64_t upc = (v8 + kClusterCtas - 1) / kClusterCtas;
+  const size_t smem = static_cast<size_t>(4 * upc * 16) + kClusterSmemExtra;
+  bool done = false;
+  if (V % 8 == 0 && smem <= 220 * 1024) {
+    err = cudaFuncSetAttribute(ear_kl_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kClusterThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kClusterCtas;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(kClusterCtas * 64, 1, 1);
+    int max_clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&max_clusters, ear_kl_cluster_kernel, &cfg) != cudaSuccess)
+      max_clusters = 0;
+    cudaGetLastError();
+    if (max_clusters > 0) {
+      const int64_t nc = T < max_clusters ? T : max_clusters;
+      cfg.gridDim = dim3(static_cast<unsigned>(kClusterCtas * nc), 1, 1);
+      err = cudaLaunchKernelEx(&cfg, ear_kl_cluster_kernel, a, b, T, V, static_cast<int>(upc), c,
+                               inv_temp, ear_tok, kl_tok, flags);
+      if (err != cudaSuccess) return err;
+      done = true;
+    }
+  }
+  if (!done) {
+    constexpr int kThreads = 1024;
+    const int64_t blocks = T < static_cast<int64_t>(sms) * 2 ? T : static_cast<int64_t>(sms) * 2;
+    if (V % 8 == 0)
+      ear_kl_rows_kernel<kThreads, true><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
+          a, b, T, V, c, inv_temp, ear_tok, kl_tok);
+    else
+      ear_kl_rows_kernel<kThreads, false><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
+          a, b, T, V, c, inv_temp, ear_tok, kl_tok);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
   if (ear_mean || kl_mean) {
     token_mean_kernel<<<1, 1024, 0, stream>>>(ear_tok, kl_tok, T, ear_mean, kl_mean);
     err = cudaGetLastError();

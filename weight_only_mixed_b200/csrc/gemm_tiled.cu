@@ -1,10 +1,630 @@
-// gemm_tiled.cu -- placeholder until the tcgen05 tiled kernel lands.
+// gemm_tiled.cu -- tiled dequantize-GEMM on the 5th-generation tensor cores.
+//
+// Y = X W^T with w = s * (q - z) (the weight-only linear layer of the pages'
+// serving path; gist.science summary, Key Results "Inference Speedup").  This
+// kernel serves M > 16 (prefill and large batches), where the contraction is
+// dense enough for the tensor cores to be the bound.
+//
+// Orientation: the weight tile is the A operand (M_mma = 128 rows of W), the
+// activation tile is the B operand (N_mma = BN rows of X, 64..256), so one
+// dequantized weight tile feeds BN activation rows and the product sits in
+// TMEM as 128 lanes (rows n of W) x BN fp32 columns (rows m of X).
+//
+// Exact scaling.  The A operand is (q - z), an integer of at most 8 bits and so
+// an exact bf16 value.  Each 128-wide group g is multiplied into its own TMEM
+// buffer P_g (two buffers, alternating), and the worker warps -- each thread
+// owns one TMEM lane, i.e. one row n of W -- add s[n, g] * P_g into fp32
+// registers.  The only rounding is fp32 accumulation, as in the decode kernel.
+//
+// Warp roles (352 threads, one CTA per 128 x BN output tile):
+//   warp 0      TMA producer of X tiles (64 k x BN rows, 128-byte swizzle).
+//   warp 1      TMEM allocator; one lane issues every tcgen05.mma.
+//   warp 2      TMA producer of packed W (one group x 128 rows per stage,
+//               swizzled so the dequant reads are conflict free); its 32 lanes
+//               also stage the group's fp16 scales and uint8 zeros.
+//   warps 3-10  dequantize group g (each lane: 32 codes of one row -> exact
+//               bf16 (q - z) in the K-major 128-byte-swizzled layout tcgen05
+//               reads), then fold P_{g-1} into the register accumulators, and
+//               finally store Y.
+// Stages are handed over with mbarriers (TMA complete_tx, tcgen05.commit and
+// plain arrivals); every wait gives up after 2 s of wall time, raises
+// SLQ_FLAG_TIMEOUT and lets the CTA drain its copies and free TMEM.
+#include <cooperative_groups.h>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
 #include "internal.h"
+#include "ptx.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace slq {
-cudaError_t launch_gemm_tiled(const uint16_t*, int64_t, int64_t, int64_t, int, const uint32_t*,
-                              const uint16_t*, const uint8_t*, void*, bool, uint32_t*,
-                              cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+
+constexpr int kBM = 128;     // W rows per tile (MMA M)
+constexpr int kBK = 64;      // k per A / X stage: one 128-byte swizzle atom of bf16
+constexpr int kSA = 4;       // dequantized A stages (two groups)
+constexpr int kSRing = 16;   // scale / zero ring (groups); must exceed packed stages + 2
+constexpr int kWorkers = 8;  // dequant + accumulate warps
+constexpr int kMaxCluster = 8;
+constexpr int kWarpX = 0, kWarpMma = 1, kWarpW = 2, kWarp0 = 3;
+constexpr int kThreads = (kWarp0 + kWorkers) * 32;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+template <int B>
+constexpr int p_stage_bytes() {
+  return kBM * 16 * B;
 }
+
+// Stage counts and the shared-memory budget.  Narrow tiles (BN <= 64, the
+// decode and small-batch shapes) aim for two CTAs per SM and spend what is
+// left of ~110 KB on packed-W stages, so that many bytes of weights are in
+// flight; wide tiles use one CTA per SM.
+template <int B, int BN>
+struct Cfg {
+  static constexpr int kSX = BN == 256 ? 3 : 4;
+  static constexpr int kXStage = BN * 128;
+  static constexpr int kAStage = kBM * 128;
+  static constexpr int kFixed = 1024 /* alignment slack */ + kSX * kXStage + kSA * kAStage +
+                                kSRing * kBM * 3 + 512 /* barriers, TMEM address, flag */;
+  static constexpr int kBudget = BN <= 64 ? 110 * 1024 : 227 * 1024;
+  static constexpr int kSPRaw = (kBudget - kFixed) / p_stage_bytes<B>();
+  static constexpr int kSP = kSPRaw > 8 ? 8 : (kSPRaw < 2 ? 2 : kSPRaw);
+  static constexpr int kSmem = kFixed + kSP * p_stage_bytes<B>();
+  static_assert(kSmem <= 232448, "shared memory budget");
+  // The producer refills scale slot g % kSRing once the dequant of group
+  // g - kSP is done, which guarantees only that the scales of groups up to
+  // g - kSP - 2 have been consumed.
+  static_assert(kSRing >= kSP + 2, "scale ring shorter than the packed-W pipeline");
+  static_assert(BN > 64 || kSA * kAStage >= kBM * BN * 4,
+                "A stages double as the split-K partial buffer");
+};
+
+// Physical byte offset of a logical offset inside a packed-W stage, for the
+// swizzle mode its tensor map uses (128/64/32-byte rows for b = 8/4/2).
+template <int B>
+__device__ __forceinline__ uint32_t p_swz(uint32_t off) {
+  if constexpr (B == 8) return off ^ (((off >> 7) & 7u) << 4);
+  else if constexpr (B == 4) return off ^ (((off >> 7) & 3u) << 4);
+  else if constexpr (B == 2) return off ^ (((off >> 7) & 1u) << 4);
+  else return off;
+}
+
+// b words (32 codes) of row `row`, unit u (codes [32u, 32u+32)) of a stage.
+template <int B>
+__device__ __forceinline__ void load_unit(const uint8_t* st, int row, int u, uint32_t (&w)[B]) {
+  if constexpr (B == 8) {
+    const uint32_t off = row * 128 + 32 * u;
+    const uint4 v0 = *reinterpret_cast<const uint4*>(st + p_swz<8>(off));
+    const uint4 v1 = *reinterpret_cast<const uint4*>(st + p_swz<8>(off + 16));
+    w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+    w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+  } else if constexpr (B == 4) {
+    const uint4 v = *reinterpret_cast<const uint4*>(st + p_swz<4>(row * 64 + 16 * u));
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  } else if constexpr (B == 2) {
+    const uint2 v = *reinterpret_cast<const uint2*>(st + p_swz<2>(row * 32 + 8 * u));
+    w[0] = v.x; w[1] = v.y;
+  } else if constexpr (B == 6) {
+    const uint8_t* p = st + row * 96 + 24 * u;
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+      const uint2 v = *reinterpret_cast<const uint2*>(p + 8 * i);
+      w[2 * i] = v.x; w[2 * i + 1] = v.y;
+    }
+  } else {
+    const uint32_t* p = reinterpret_cast<const uint32_t*>(st + row * 16 * B + 4 * B * u);
+#pragma unroll
+    for (int i = 0; i < B; ++i) w[i] = p[i];
+  }
+}
+
+template <int B>
+__device__ __forceinline__ uint32_t code_at(const uint32_t (&w)[B], int i) {
+  const int o = B * i;
+  const int wi = o >> 5;
+  const int sh = o & 31;
+  constexpr uint32_t mask = (1u << B) - 1u;
+  if (sh + B <= 32) return (w[wi] >> sh) & mask;
+  return __funnelshift_r(w[wi], w[wi + 1], sh) & mask;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a),
+                             *reinterpret_cast<__nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// The 32 codes of a unit as 16 bf16x2 registers (q_{2p} - z, q_{2p+1} - z),
+// consecutive k, exact.  For b <= 7 each code is ORed into the mantissa of
+// bf16 128.0 and (128 + z) is subtracted in bf16; b = 8 goes through binary32
+// (2^23 + q) - (2^23 + z).  For b = 4 and b = 2 one byte is isolated with a
+// byte permute and a multiply by 0x1001 / 0x4001 places its two codes 16 bits
+// apart, so a single AND/OR forms the pair.
+template <int B>
+__device__ __forceinline__ void unit_pairs(const uint32_t (&w)[B], uint32_t z, uint32_t (&out)[16]) {
+  if constexpr (B == 8) {
+    const float zf = __uint_as_float(0x4B000000u | z);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float lo = __uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7540 | (2 * h)));
+        const float hi = __uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7540 | (2 * h + 1)));
+        __nv_bfloat162 v = __floats2bfloat162_rn(__fsub_rn(lo, zf), __fsub_rn(hi, zf));
+        out[2 * i + h] = *reinterpret_cast<uint32_t*>(&v);
+      }
+    }
+  } else {
+    const uint32_t z2 = (0x4300u | z) * 0x00010001u;  // bf16x2 (128 + z, 128 + z)
+    if constexpr (B == 4) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t y = __byte_perm(w[i], 0u, 0x4440 | k) * 0x1001u;
+          out[4 * i + k] = bf16x2_sub((y & 0x000F000Fu) | 0x43004300u, z2);
+        }
+    } else if constexpr (B == 2) {
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t y = __byte_perm(w[i], 0u, 0x4440 | k) * 0x4001u;
+          out[8 * i + 2 * k] = bf16x2_sub((y & 0x00030003u) | 0x43004300u, z2);
+          out[8 * i + 2 * k + 1] = bf16x2_sub(((y >> 4) & 0x00030003u) | 0x43004300u, z2);
+        }
+    } else {
+#pragma unroll
+      for (int p = 0; p < 16; ++p)
+        out[p] = bf16x2_sub(code_at<B>(w, 2 * p) | (code_at<B>(w, 2 * p + 1) << 16) | 0x43004300u, z2);
+    }
+  }
+}
+
+// UMMA shared-memory descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (SBO), descriptor version 1 (sm_100).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
+         (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+         (static_cast<uint64_t>(2) << 61);
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B (K-major), fp32 D, M = 128, N = BN.
+template <int BN>
+__host__ __device__ constexpr uint32_t instr_desc() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
+         (static_cast<uint32_t>(kBM >> 4) << 24);
+}
+
+struct Bars {
+  uint64_t* x_full;
+  uint64_t* x_empty;
+  uint64_t* a_full;
+  uint64_t* a_empty;
+  uint64_t* p_full;
+  uint64_t* p_empty;
+  uint64_t* pf;  // P buffer filled (tcgen05.commit)
+  uint64_t* pe;  // P buffer drained by the workers
+  uint64_t* mma_done;
+  uint32_t* tmem_base;
+  volatile int* abort_flag;
+};
+
+// Bounded wait; on timeout raises the flag word and the CTA-wide abort flag.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, const Bars& sh,
+                                              uint32_t* flags) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*sh.abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *sh.abort_flag = 1;
+      if (flags) atomicOr(flags, kFlagTimeout);
+      return false;
+    }
+  }
+}
+
+template <int B, int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                      const __grid_constant__ CUtensorMap tmap_w, int M, int N, int K,
+                      const uint16_t* __restrict__ scales, const uint8_t* __restrict__ zeros,
+                      void* __restrict__ Y, int y_f32, int groups_per_slice,
+                      uint32_t* __restrict__ flags) {
+  using C = Cfg<B, BN>;
+  constexpr int kSP = C::kSP;
+  constexpr int kCols = 2 * BN;  // two P buffers
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* xbuf = smem;
+  uint8_t* abuf = xbuf + C::kSX * C::kXStage;
+  uint8_t* pbuf = abuf + kSA * C::kAStage;
+  uint16_t* sring = reinterpret_cast<uint16_t*>(pbuf + kSP * p_stage_bytes<B>());  // [kSRing][128]
+  uint8_t* zring = reinterpret_cast<uint8_t*>(sring + kSRing * kBM);                // [kSRing][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(zring + kSRing * kBM);
+  Bars sh;
+  sh.x_full = bars;
+  sh.x_empty = sh.x_full + C::kSX;
+  sh.a_full = sh.x_empty + C::kSX;
+  sh.a_empty = sh.a_full + kSA;
+  sh.p_full = sh.a_empty + kSA;
+  sh.p_empty = sh.p_full + kSP;
+  sh.pf = sh.p_empty + kSP;
+  sh.pe = sh.pf + 2;
+  sh.mma_done = sh.pe + 2;
+  sh.tmem_base = reinterpret_cast<uint32_t*>(sh.mma_done + 1);
+  sh.abort_flag = reinterpret_cast<volatile int*>(sh.tmem_base + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * kBM;
+  const int m0 = blockIdx.y * BN;
+  const int G = K / kGroup;
+  // K slice of this CTA (blockIdx.z; the CTAs of one slice set form a cluster).
+  const int g_begin = blockIdx.z * groups_per_slice;
+  const int g_end = min(G, g_begin + groups_per_slice);
+  const int ng = g_end - g_begin;
+  const int KB = 2 * ng;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kSX; ++i) {
+      mbar_init(&sh.x_full[i], 1);
+      mbar_init(&sh.x_empty[i], 1);
+    }
+    for (int i = 0; i < kSA; ++i) {
+      mbar_init(&sh.a_full[i], kWorkers);
+      mbar_init(&sh.a_empty[i], 1);
+    }
+    for (int i = 0; i < kSP; ++i) {
+      mbar_init(&sh.p_full[i], 1 + 32);  // TMA arrival + the producer warp's lanes
+      mbar_init(&sh.p_empty[i], kWorkers);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh.pf[i], 1);
+      mbar_init(&sh.pe[i], kWorkers);
+    }
+    mbar_init(sh.mma_done, 1);
+    *sh.abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncwarp();
+  if (warp == kWarpMma) {
+    tmem_alloc(sh.tmem_base, kCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *sh.tmem_base;
+
+  if (warp == kWarpX) {
+    // ---------------- X producer ----------------
+    if (lane == 0) {
+      prefetch_tmap(&tmap_x);
+      int issued = 0;
+      for (int kb = 0; kb < KB; ++kb) {
+        const int s = kb % C::kSX;
+        if (!wait_or_abort(&sh.x_empty[s], ((kb / C::kSX) & 1) ^ 1, sh, flags)) break;
+        mbar_arrive_expect_tx(&sh.x_full[s], C::kXStage);
+        tma_load_2d(xbuf + s * C::kXStage, &tmap_x, &sh.x_full[s], (2 * g_begin + kb) * kBK, m0);
+        ++issued;
+      }
+      // Drain: every issued copy must land before the CTA may exit.
+      for (int i = issued - C::kSX; i < issued; ++i)
+        if (i >= 0) mbar_wait_bounded(&sh.x_full[i % C::kSX], (i / C::kSX) & 1, kWaitLimitNs);
+    }
+    __syncwarp();
+  } else if (warp == kWarpW) {
+    // ---------------- packed-W producer + scale / zero staging ----------------
+    // Lane l stages rows 4l..4l+3.  The scale / zero loads run kLookahead
+    // groups ahead of the stores (a register pipeline), so their DRAM latency
+    // overlaps the ring instead of stalling every group.
+    if (lane == 0) prefetch_tmap(&tmap_w);
+    constexpr int kLookahead = BN <= 64 ? 8 : 4;
+    auto fetch = [&](int g, int q) -> uint32_t {
+      const int n = n0 + 4 * lane + q;
+      if (g >= ng || n >= N) return 0u;
+      const int64_t gi = static_cast<int64_t>(n) * G + g_begin + g;
+      return static_cast<uint32_t>(scales[gi]) | (static_cast<uint32_t>(zeros[gi]) << 16);
+    };
+    uint32_t pipe[kLookahead][4];
+#pragma unroll
+    for (int j = 0; j < kLookahead; ++j)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) pipe[j][q] = fetch(j, q);
+    int issued = 0;
+    for (int g = 0; g < ng; ++g) {
+      const int s = g % kSP;
+      const bool ok = wait_or_abort(&sh.p_empty[s], ((g / kSP) & 1) ^ 1, sh, flags);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&sh.p_full[s], p_stage_bytes<B>());
+        tma_load_2d(pbuf + s * p_stage_bytes<B>(), &tmap_w, &sh.p_full[s], (g_begin + g) * 4 * B, n0);
+      }
+      uint16_t* sr = sring + (g % kSRing) * kBM;
+      uint8_t* zr = zring + (g % kSRing) * kBM;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        sr[4 * lane + q] = static_cast<uint16_t>(pipe[0][q] & 0xFFFFu);
+        zr[4 * lane + q] = static_cast<uint8_t>(pipe[0][q] >> 16);
+      }
+      mbar_arrive(&sh.p_full[s]);
+      ++issued;
+#pragma unroll
+      for (int j = 0; j < kLookahead - 1; ++j)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) pipe[j][q] = pipe[j + 1][q];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) pipe[kLookahead - 1][q] = fetch(g + kLookahead, q);
+    }
+    if (lane == 0)
+      for (int i = issued - kSP; i < issued; ++i)
+        if (i >= 0) mbar_wait_bounded(&sh.p_full[i % kSP], (i / kSP) & 1, kWaitLimitNs);
+    __syncwarp();
+  } else if (warp == kWarpMma) {
+    // ---------------- MMA issuer: group g into P[g % 2] ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = instr_desc<BN>();
+      bool ok = true;
+      for (int g = 0; g < ng && ok; ++g) {
+        const int buf = g & 1;
+        ok = wait_or_abort(&sh.pe[buf], ((g >> 1) & 1) ^ 1, sh, flags);
+        if (!ok) break;
+        tc_fence_after_sync();
+        const uint32_t d = tmem + static_cast<uint32_t>(buf * BN);
+#pragma unroll 1
+        for (int h = 0; h < 2 && ok; ++h) {
+          const int kb = 2 * g + h;
+          const int sa = kb % kSA, sx = kb % C::kSX;
+          ok = wait_or_abort(&sh.a_full[sa], (kb / kSA) & 1, sh, flags) &&
+               wait_or_abort(&sh.x_full[sx], (kb / C::kSX) & 1, sh, flags);
+          if (!ok) break;
+          tc_fence_after_sync();
+          const uint64_t da = sw128_desc(smem_u32(abuf + sa * C::kAStage));
+          const uint64_t db = sw128_desc(smem_u32(xbuf + sx * C::kXStage));
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k)  // +32 bytes along K per MMA: +2 in the address field
+            umma_bf16_ss(d, da + 2 * k, db + 2 * k, idesc, (h > 0 || k > 0) ? 1u : 0u);
+          umma_commit(&sh.a_empty[sa]);
+          umma_commit(&sh.x_empty[sx]);
+        }
+        if (ok) umma_commit(&sh.pf[buf]);
+      }
+      umma_commit(sh.mma_done);
+      mbar_wait_bounded(sh.mma_done, 0, kWaitLimitNs);  // no MMA in flight past this point
+    }
+    __syncwarp();
+  } else {
+    // ---------------- workers ----------------
+    const int d = warp - kWarp0;  // dequant rows [16d, 16d + 16)
+    const int u = lane >> 3;      // dequant unit: codes [32u, 32u + 32) of the group
+    const int q = warp & 3;       // TMEM lane quarter this warp may access
+    const int hcol = d >> 2;      // accumulator column half
+    constexpr int kHalf = BN / 2;
+    float acc[kHalf];
+#pragma unroll
+    for (int j = 0; j < kHalf; ++j) acc[j] = 0.0f;
+
+    bool ok = true;
+    for (int g = 0; g <= ng && ok; ++g) {
+      if (g < ng) {
+        // ---- dequantize group g into A stages 2g, 2g+1 ----
+        const int sp = g % kSP;
+        ok = wait_or_abort(&sh.a_empty[(2 * g) % kSA], (((2 * g) / kSA) & 1) ^ 1, sh, flags) &&
+             wait_or_abort(&sh.a_empty[(2 * g + 1) % kSA], (((2 * g + 1) / kSA) & 1) ^ 1, sh, flags) &&
+             wait_or_abort(&sh.p_full[sp], (g / kSP) & 1, sh, flags);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        const uint8_t* pst = pbuf + sp * p_stage_bytes<B>();
+        const uint8_t* zr = zring + (g % kSRing) * kBM;
+#pragma unroll
+        for (int it = 0; it < 2; ++it) {
+          const int row = 16 * d + 8 * it + (lane & 7);
+          const uint32_t z = zr[row];
+          uint32_t w[B];
+          load_unit<B>(pst, row, u, w);
+          uint32_t pr[16];
+          unit_pairs<B>(w, z, pr);
+          uint8_t* ast = abuf + ((2 * g + (u >> 1)) % kSA) * C::kAStage + row * 128;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int chunk = ((u & 1) * 4 + c) ^ (row & 7);
+            *reinterpret_cast<uint4*>(ast + chunk * 16) =
+                make_uint4(pr[4 * c], pr[4 * c + 1], pr[4 * c + 2], pr[4 * c + 3]);
+          }
+        }
+        fence_proxy_async_smem();  // generic-proxy smem writes -> visible to tcgen05.mma
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&sh.a_full[(2 * g) % kSA]);
+          mbar_arrive(&sh.a_full[(2 * g + 1) % kSA]);
+          mbar_arrive(&sh.p_empty[sp]);
+        }
+      }
+      if (g >= 1) {
+        // ---- fold P_{g-1} into the accumulators: acc += s[n, g-1] * P ----
+        const int j = g - 1;
+        const int buf = j & 1;
+        ok = __all_sync(0xffffffffu, wait_or_abort(&sh.pf[buf], (j >> 1) & 1, sh, flags));
+        if (!ok) break;
+        tc_fence_after_sync();
+        const float s =
+            __half2float(__ushort_as_half(sring[(j % kSRing) * kBM + 32 * q + lane]));
+        const uint32_t base = tmem + (static_cast<uint32_t>(32 * q) << 16) +
+                              static_cast<uint32_t>(buf * BN + hcol * kHalf);
+        if constexpr (kHalf % 16 == 0) {
+#pragma unroll
+          for (int c = 0; c < kHalf / 16; ++c) {
+            uint32_t r[16];
+            tmem_ld_32x32b_x16(base + 16 * c, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) acc[16 * c + i] = fmaf(s, __uint_as_float(r[i]), acc[16 * c + i]);
+          }
+        } else {
+          uint32_t r[8];
+          tmem_ld_32x32b_x8(base, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] = fmaf(s, __uint_as_float(r[i]), acc[i]);
+        }
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.pe[buf]);
+      }
+    }
+
+    // ---- epilogue: thread owns row n, columns m0 + hcol * BN/2 + [0, BN/2) ----
+    if (gridDim.z > 1) {
+      // Split K: partial sums go to shared memory (the A stages are idle now:
+      // every MMA has completed), the cluster adds them up below.
+      float* part = reinterpret_cast<float*>(abuf);
+#pragma unroll
+      for (int j = 0; j < kHalf; ++j) part[(hcol * kHalf + j) * kBM + 32 * q + lane] = acc[j];
+    } else if (ok) {
+      const int n = n0 + 32 * q + lane;
+      if (n < N) {
+#pragma unroll
+        for (int j = 0; j < kHalf; ++j) {
+          const int m = m0 + hcol * kHalf + j;
+          if (m < M) {
+            const int64_t o = static_cast<int64_t>(m) * N + n;
+            if (y_f32)
+              static_cast<float*>(Y)[o] = acc[j];
+            else
+              static_cast<__nv_bfloat16*>(Y)[o] = __float2bfloat16_rn(acc[j]);
+          }
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  if (gridDim.z > 1) {
+    // Cross-CTA reduction over the K slices of the cluster, in rank order
+    // (deterministic; no atomics, no global workspace).
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();  // every CTA's partial sums are complete and visible
+    if (cluster.block_rank() == 0) {
+      const float* part = reinterpret_cast<const float*>(abuf);
+      const int nz = static_cast<int>(gridDim.z);
+      for (int e = threadIdx.x; e < kBM * BN; e += kThreads) {
+        float v = part[e];
+        for (int c = 1; c < nz; ++c) v += cluster.map_shared_rank(part, c)[e];
+        const int n = n0 + e % kBM, m = m0 + e / kBM;
+        if (n < N && m < M) {
+          const int64_t o = static_cast<int64_t>(m) * N + n;
+          if (y_f32)
+            static_cast<float*>(Y)[o] = v;
+          else
+            static_cast<__nv_bfloat16*>(Y)[o] = __float2bfloat16_rn(v);
+        }
+      }
+    }
+    cluster.sync();  // keep every CTA's shared memory alive until rank 0 has read it
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+template <int B, int BN>
+cudaError_t launch_cfg(const uint16_t* X, int M, int N, int K, const uint32_t* packed,
+                       const uint16_t* scales, const uint8_t* zeros, void* Y, bool y_f32,
+                       uint32_t* flags, cudaStream_t stream) {
+  using C = Cfg<B, BN>;
+  CUtensorMap tx, tw;
+  const CUtensorMapSwizzle swz = B == 8   ? CU_TENSOR_MAP_SWIZZLE_128B
+                                 : B == 4 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                 : B == 2 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                          : CU_TENSOR_MAP_SWIZZLE_NONE;
+  if (!encode_tensor_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, static_cast<uint64_t>(K),
+                            static_cast<uint64_t>(M), static_cast<uint64_t>(K) * 2, kBK, BN,
+                            CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tensor_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, packed,
+                            static_cast<uint64_t>(K) * B / 32, static_cast<uint64_t>(N),
+                            static_cast<uint64_t>(K) * B / 8, 4 * B, kBM, swz))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(gemm_tiled_kernel<B, BN>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int G = K / kGroup;
+  const int row_blocks = (N + kBM - 1) / kBM;
+  const int col_blocks = (M + BN - 1) / BN;
+  // Narrow tiles: split K over a cluster so that the CTAs fill the resident
+  // slots (two per SM) in one wave without spilling into a second one; each
+  // slice keeps at least four groups.
+  int C_split = 1;
+  if (BN <= 64) {
+    const int tiles = row_blocks * col_blocks;
+    C_split = (2 * sms) / tiles;
+    if (C_split > kMaxCluster) C_split = kMaxCluster;
+    if (C_split > G / 4) C_split = G / 4;
+    if (C_split < 1) C_split = 1;
+  }
+  const int per_slice = (G + C_split - 1) / C_split;
+  C_split = (G + per_slice - 1) / per_slice;  // no empty slices
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(row_blocks), static_cast<unsigned>(col_blocks),
+                     static_cast<unsigned>(C_split));
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = static_cast<unsigned>(C_split);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_tiled_kernel<B, BN>, tx, tw, M, N, K, scales, zeros, Y,
+                            y_f32 ? 1 : 0, per_slice, flags);
+}
+
+// Tile width: BN = 16 for decode batches (M <= 16), otherwise the smallest of
+// 64 / 128 / 256 that covers M, so padding rows cost no more than needed.
+template <int B>
+cudaError_t launch_b(const uint16_t* X, int M, int N, int K, const uint32_t* packed,
+                     const uint16_t* scales, const uint8_t* zeros, void* Y, bool y_f32,
+                     bool decode, uint32_t* flags, cudaStream_t stream) {
+  if (decode) return launch_cfg<B, 16>(X, M, N, K, packed, scales, zeros, Y, y_f32, flags, stream);
+  if (M <= 64) return launch_cfg<B, 64>(X, M, N, K, packed, scales, zeros, Y, y_f32, flags, stream);
+  if (M <= 128) return launch_cfg<B, 128>(X, M, N, K, packed, scales, zeros, Y, y_f32, flags, stream);
+  return launch_cfg<B, 256>(X, M, N, K, packed, scales, zeros, Y, y_f32, flags, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_tiled(const uint16_t* X, int64_t M, int64_t N, int64_t K, int bits,
+                              const uint32_t* packed, const uint16_t* scales, const uint8_t* zeros,
+                              void* Y, bool y_f32, bool decode, uint32_t* flags,
+                              cudaStream_t stream) {
+  const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
+  switch (bits) {
+    case 2: return launch_b<2>(X, m, n, k, packed, scales, zeros, Y, y_f32, decode, flags, stream);
+    case 3: return launch_b<3>(X, m, n, k, packed, scales, zeros, Y, y_f32, decode, flags, stream);
+    case 4: return launch_b<4>(X, m, n, k, packed, scales, zeros, Y, y_f32, decode, flags, stream);
+    case 5: return launch_b<5>(X, m, n, k, packed, scales, zeros, Y, y_f32, decode, flags, stream);
+    case 6: return launch_b<6>(X, m, n, k, packed, scales, zeros, Y, y_f32, decode, flags, stream);
+    case 7: return launch_b<7>(X, m, n, k, packed, scales, zeros, Y, y_f32, decode, flags, stream);
+    case 8: return launch_b<8>(X, m, n, k, packed, scales, zeros, Y, y_f32, decode, flags, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 }  // namespace slq

@@ -2,6 +2,7 @@
 // the kernel translation units.  Not part of the public ABI (see include/slq.h).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -18,18 +19,18 @@ cudaError_t launch_quantize(const uint16_t* W, int64_t N, int64_t K, int bits,
                             uint32_t* packed, uint16_t* scales, uint8_t* zeros,
                             uint32_t* flags, cudaStream_t stream);
 
-// Decode GEMV/skinny GEMM for M <= 16 (register dequant + mma.sync).
-cudaError_t launch_gemm_decode(const uint16_t* X, int64_t M, int64_t N, int64_t K,
-                               int bits, const uint32_t* packed,
-                               const uint16_t* scales, const uint8_t* zeros,
-                               void* Y, bool y_f32, cudaStream_t stream);
+// Encode a 2-D tiled TMA map (inner dimension contiguous); false on failure.
+bool encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                          uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
+                          uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
-// Tiled GEMM (TMA + dequant-to-smem + tcgen05.mma with TMEM accumulators).
-cudaError_t launch_gemm_tiled(const uint16_t* X, int64_t M, int64_t N, int64_t K,
-                              int bits, const uint32_t* packed,
-                              const uint16_t* scales, const uint8_t* zeros,
-                              void* Y, bool y_f32, uint32_t* flags,
-                              cudaStream_t stream);
+// Dequantize-GEMM on tcgen05 (TMA + dequant to shared memory + tcgen05.mma
+// with TMEM accumulators).  decode = true selects the 16-wide activation tile
+// with split-K over a cluster (M <= 16); otherwise the tile width follows M.
+cudaError_t launch_gemm_tiled(const uint16_t* X, int64_t M, int64_t N, int64_t K, int bits,
+                              const uint32_t* packed, const uint16_t* scales,
+                              const uint8_t* zeros, void* Y, bool y_f32, bool decode,
+                              uint32_t* flags, cudaStream_t stream);
 
 cudaError_t launch_ear_kl(const uint16_t* a, const uint16_t* b, int64_t T, int64_t V,
                           float temperature, float* ear_tok, float* kl_tok,
