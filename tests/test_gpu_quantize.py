@@ -96,3 +96,29 @@ def test_full_size_sampled_rows(N, K, bits):
     assert np.array_equal(to_host_u16(qw.scales.index_select(0, idx)), want[1])
     assert np.array_equal(qw.zeros.index_select(0, idx).cpu().numpy(), want[2])
     assert np.array_equal(to_host_u32(qw.packed.index_select(0, idx)), want[0])
+
+
+def _near_tie_groups(bits: int, n_groups: int = 96, seed: int = 0) -> np.ndarray:
+    """Groups whose elements sit exactly on half-integer multiples of the step,
+    or one bf16 ulp to either side: the cases where a quotient computed any
+    other way than the IEEE division would round differently."""
+    rng = np.random.default_rng(seed + bits)
+    maxq = 2**bits - 1
+    rows = []
+    for _ in range(n_groups):
+        e = int(rng.integers(-12, 5))
+        s = 2.0**e
+        k = rng.integers(0, min(maxq, 127), size=126)
+        v = (k + 0.5) * s
+        bits16 = synth.to_bf16_bits(v)
+        nudge = rng.integers(-1, 2, size=126).astype(np.int32)  # -1, 0, +1 ulp
+        bits16 = (bits16.astype(np.int32) + nudge).astype(np.uint16)
+        vals = synth.bf16_bits_to_f32(bits16).astype(np.float64)
+        g = np.concatenate([[0.0, maxq * s], vals])  # pins the range: scale = s exactly
+        rows.append(g)
+    return synth.to_bf16_bits(np.array(rows).reshape(1, -1))
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_near_ties_are_bit_exact(bits):
+    _assert_same(_near_tie_groups(bits), bits)

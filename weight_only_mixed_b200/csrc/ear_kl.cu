@@ -215,80 +215,33 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // ---------------------------------------------------------------------------
-// Cluster kernel (V % 8 == 0): one HBM pass.  A cluster of 8 CTAs owns one
-// token row at a time; CTA r keeps slice r of both logit rows in shared memory
-// (double-buffered 1-D bulk copies, the next row lands while this one is
-// processed).  Per row: local max, local sums -> statistics exchanged through
-// distributed shared memory and merged in rank order -> the EAR sum from the
-// resident slice.  The EAR partials of row i are added up by rank 0 after the
-// exchange of row i+1, so each row costs a single cluster barrier.
+// Cluster kernel (V % 8 == 0): one HBM pass.  A cluster of CS CTAs (8, or 16
+// where the GPU allows it) owns one token row at a time; CTA r keeps slice r
+// of both logit rows in shared memory (double-buffered 1-D bulk copies: the
+// next row lands while this one is processed).  Per row: one pass of online
+// softmax statistics (running max with rescaling) -> one block reduction ->
+// the statistics are exchanged through distributed shared memory and merged
+// in rank order -> the EAR sum over the resident slice.  Rank 0 adds the EAR
+// partials of row i after the exchange of row i+1, so each row costs a single
+// cluster barrier.
 // ---------------------------------------------------------------------------
-constexpr int kClusterCtas = 8;
 constexpr int kClusterThreads = 512;
 
 struct SliceStat {
   float ma, sa, w, mb, sb;
 };
 
-template <int kThreads>
-__device__ float2 block_max2(float x, float y, float* red) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    x = fmaxf(x, __shfl_xor_sync(kFull, x, off));
-    y = fmaxf(y, __shfl_xor_sync(kFull, y, off));
-  }
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (lane == 0) {
-    red[2 * warp] = x;
-    red[2 * warp + 1] = y;
-  }
-  __syncthreads();
-  float rx = red[0], ry = red[1];
-  for (int w = 1; w < kThreads / 32; ++w) {
-    rx = fmaxf(rx, red[2 * w]);
-    ry = fmaxf(ry, red[2 * w + 1]);
-  }
-  __syncthreads();
-  return make_float2(rx, ry);
-}
-
-// Sum of three values over the block, fixed order; valid in every thread.
-template <int kThreads>
-__device__ float3 block_sum3(float x, float y, float z, float* red) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    x += __shfl_xor_sync(kFull, x, off);
-    y += __shfl_xor_sync(kFull, y, off);
-    z += __shfl_xor_sync(kFull, z, off);
-  }
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (lane == 0) {
-    red[3 * warp] = x;
-    red[3 * warp + 1] = y;
-    red[3 * warp + 2] = z;
-  }
-  __syncthreads();
-  float rx = 0.0f, ry = 0.0f, rz = 0.0f;
-  for (int w = 0; w < kThreads / 32; ++w) {
-    rx += red[3 * w];
-    ry += red[3 * w + 1];
-    rz += red[3 * w + 2];
-  }
-  __syncthreads();
-  return make_float3(rx, ry, rz);
-}
-
-__global__ void __launch_bounds__(kClusterThreads, 1)
+template <int CS>
+__global__ void __launch_bounds__(kClusterThreads)
     ear_kl_cluster_kernel(const uint16_t* __restrict__ A, const uint16_t* __restrict__ Bq,
                           int64_t T, int64_t V, int units_per_cta, float c, float inv_temp,
                           float* __restrict__ ear_tok, float* __restrict__ kl_tok,
                           uint32_t* __restrict__ flags) {
-  constexpr uint64_t kWaitLimitNs = 2000000000ull;
   extern __shared__ __align__(128) uint8_t smem[];
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
-  const int64_t cluster_id = blockIdx.x / kClusterCtas;
-  const int64_t nclusters = gridDim.x / kClusterCtas;
+  const int64_t cluster_id = blockIdx.x / CS;
+  const int64_t nclusters = gridDim.x / CS;
 
   const int64_t v8 = V / 8;
   const int64_t r0 = static_cast<int64_t>(rank) * units_per_cta;
@@ -297,13 +250,12 @@ __global__ void __launch_bounds__(kClusterThreads, 1)
   const int nu = static_cast<int>(u1 - u0);  // 16-byte units of this CTA's slice
   const size_t slice_bytes = static_cast<size_t>(units_per_cta) * 16;
 
-  // [buf][tensor][slice] | barriers | stats[2] | ear[2] | merged | reduction scratch
+  // [buf][tensor][slice] | barriers | stats[2] | ear[2] | merged
   uint8_t* data = smem;
   uint64_t* full = reinterpret_cast<uint64_t*>(data + 4 * slice_bytes);
   SliceStat* stats = reinterpret_cast<SliceStat*>(full + 2);
   float* ear_part = reinterpret_cast<float*>(stats + 2);
   SliceStat* merged = reinterpret_cast<SliceStat*>(ear_part + 2);
-  float* red = reinterpret_cast<float*>(merged + 1);
   __shared__ int aborted;
 
   const int64_t nrows = (T > cluster_id) ? (T - cluster_id + nclusters - 1) / nclusters : 0;
@@ -320,25 +272,22 @@ __global__ void __launch_bounds__(kClusterThreads, 1)
   auto issue = [&](int64_t i) {
     const int buf = static_cast<int>(i & 1);
     const int64_t t = cluster_id + i * nclusters;
-    uint8_t* da = data + (2 * buf) * slice_bytes;
-    uint8_t* db = data + (2 * buf + 1) * slice_bytes;
     const uint32_t bytes = static_cast<uint32_t>(nu) * 16;
     mbar_arrive_expect_tx(&full[buf], 2 * bytes);
     if (bytes) {
-      bulk_load(da, A + t * V + u0 * 8, bytes, &full[buf]);
-      bulk_load(db, Bq + t * V + u0 * 8, bytes, &full[buf]);
+      bulk_load(data + (2 * buf) * slice_bytes, A + t * V + u0 * 8, bytes, &full[buf]);
+      bulk_load(data + (2 * buf + 1) * slice_bytes, Bq + t * V + u0 * 8, bytes, &full[buf]);
     }
   };
   int64_t issued = 0;
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0)
     for (; issued < 2 && issued < nrows; ++issued) issue(issued);
-  }
 
   for (int64_t i = 0; i < nrows; ++i) {
     const int buf = static_cast<int>(i & 1);
     const int64_t t = cluster_id + i * nclusters;
     if (!aborted) {
-      if (!mbar_wait_bounded(&full[buf], static_cast<uint32_t>((i >> 1) & 1), kWaitLimitNs)) {
+      if (!mbar_wait_bounded(&full[buf], static_cast<uint32_t>((i >> 1) & 1))) {
         aborted = 1;
         if (flags) atomicOr(flags, kFlagTimeout);
       }
@@ -348,8 +297,8 @@ __global__ void __launch_bounds__(kClusterThreads, 1)
     const uint4* sa4 = reinterpret_cast<const uint4*>(data + (2 * buf) * slice_bytes);
     const uint4* sb4 = reinterpret_cast<const uint4*>(data + (2 * buf + 1) * slice_bytes);
 
-    // Local maxima of the raw logits (the temperature scale is monotone).
-    float mxa = -INFINITY, mxb = -INFINITY;
+    // One pass of online softmax statistics over the resident slice.
+    RowStat st{{-INFINITY, 0.0f}, {-INFINITY, 0.0f}, 0.0f};
     if (live) {
       for (int k = threadIdx.x; k < nu; k += kClusterThreads) {
         const uint4 va = sa4[k], vb = sb4[k];
@@ -357,78 +306,50 @@ __global__ void __launch_bounds__(kClusterThreads, 1)
         const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          mxa = fmaxf(mxa, fmaxf(bf16_lo(wa[q]), bf16_hi(wa[q])));
-          mxb = fmaxf(mxb, fmaxf(bf16_lo(wb[q]), bf16_hi(wb[q])));
+          push(st, bf16_lo(wa[q]), bf16_lo(wb[q]), c);
+          push(st, bf16_hi(wa[q]), bf16_hi(wb[q]), c);
         }
       }
     }
-    const float2 mx = block_max2<kClusterThreads>(mxa, mxb, red);
-    // Local sums around the local maxima.
-    float s_a = 0.0f, s_b = 0.0f, w_ab = 0.0f;
-    if (live && nu > 0) {
-      for (int k = threadIdx.x; k < nu; k += kClusterThreads) {
-        const uint4 va = sa4[k], vb = sb4[k];
-        const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
-        const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float a0 = bf16_lo(wa[q]), a1 = bf16_hi(wa[q]);
-          const float b0 = bf16_lo(wb[q]), b1 = bf16_hi(wb[q]);
-          const float e0 = ex2((a0 - mx.x) * c), e1 = ex2((a1 - mx.x) * c);
-          s_a += e0 + e1;
-          w_ab = fmaf(e0, a0 - b0, fmaf(e1, a1 - b1, w_ab));
-          s_b += ex2((b0 - mx.y) * c) + ex2((b1 - mx.y) * c);
-        }
-      }
-    }
-    const float3 sums = block_sum3<kClusterThreads>(s_a, s_b, w_ab, red);
-    if (threadIdx.x == 0) stats[buf] = SliceStat{mx.x, sums.x, sums.z, mx.y, sums.y};
+    const RowStat tot = block_reduce<kClusterThreads>(st, c);
+    if (threadIdx.x == 0) stats[buf] = SliceStat{tot.a.m, tot.a.s, tot.w, tot.b.m, tot.b.s};
 
     cluster.sync();  // statistics of row i (and EAR partials of row i-1) are visible
 
     if (threadIdx.x < 32) {
-      // Merge the 8 slices in rank order (lane 0 does the fixed-order sums).
+      // Merge the CS slices in rank order (lane 0 does the fixed-order sums).
       SliceStat r = {-INFINITY, 0.0f, 0.0f, -INFINITY, 0.0f};
-      if (threadIdx.x < kClusterCtas) r = cluster.map_shared_rank(stats, static_cast<int>(threadIdx.x))[buf];
+      if (threadIdx.x < CS) r = cluster.map_shared_rank(stats, static_cast<int>(threadIdx.x))[buf];
       float prev_ear = 0.0f;
-      if (rank == 0 && i > 0 && threadIdx.x < kClusterCtas)
+      if (rank == 0 && i > 0 && threadIdx.x < CS)
         prev_ear = cluster.map_shared_rank(ear_part, static_cast<int>(threadIdx.x))[buf ^ 1];
-      SliceStat all[kClusterCtas];
-      float pe[kClusterCtas];
+      float Ma = -INFINITY, Mb = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < kClusterCtas; ++j) {
-        all[j].ma = __shfl_sync(kFull, r.ma, j);
-        all[j].sa = __shfl_sync(kFull, r.sa, j);
-        all[j].w = __shfl_sync(kFull, r.w, j);
-        all[j].mb = __shfl_sync(kFull, r.mb, j);
-        all[j].sb = __shfl_sync(kFull, r.sb, j);
-        pe[j] = __shfl_sync(kFull, prev_ear, j);
+      for (int j = 0; j < CS; ++j) {
+        Ma = fmaxf(Ma, __shfl_sync(kFull, r.ma, j));
+        Mb = fmaxf(Mb, __shfl_sync(kFull, r.mb, j));
+      }
+      float Sa = 0.0f, Sb = 0.0f, W = 0.0f, E = 0.0f;
+#pragma unroll
+      for (int j = 0; j < CS; ++j) {
+        const float ma = __shfl_sync(kFull, r.ma, j), mb = __shfl_sync(kFull, r.mb, j);
+        const float sa = __shfl_sync(kFull, r.sa, j), sb = __shfl_sync(kFull, r.sb, j);
+        const float w = __shfl_sync(kFull, r.w, j);
+        E += __shfl_sync(kFull, prev_ear, j);
+        if (ma != -INFINITY) {
+          const float f = ex2((ma - Ma) * c);
+          Sa = fmaf(sa, f, Sa);
+          W = fmaf(w, f, W);
+        }
+        if (mb != -INFINITY) Sb = fmaf(sb, ex2((mb - Mb) * c), Sb);
       }
       if (threadIdx.x == 0) {
-        float Ma = -INFINITY, Mb = -INFINITY;
-        for (int j = 0; j < kClusterCtas; ++j) {
-          Ma = fmaxf(Ma, all[j].ma);
-          Mb = fmaxf(Mb, all[j].mb);
-        }
-        float Sa = 0.0f, Sb = 0.0f, W = 0.0f;
-        for (int j = 0; j < kClusterCtas; ++j) {
-          if (all[j].ma != -INFINITY) {
-            const float f = ex2((all[j].ma - Ma) * c);
-            Sa = fmaf(all[j].sa, f, Sa);
-            W = fmaf(all[j].w, f, W);
-          }
-          if (all[j].mb != -INFINITY) Sb = fmaf(all[j].sb, ex2((all[j].mb - Mb) * c), Sb);
-        }
         *merged = SliceStat{Ma, Sa, W, Mb, Sb};
         if (rank == 0) {
           constexpr float kLn2 = 0.693147180559945309f;
-          const float la = lg2(Sa), lb = lg2(Sb);
-          if (live) kl_tok[t] = (W / Sa) * inv_temp - ((Ma - Mb) * inv_temp + (la - lb) * kLn2);
-          if (i > 0) {
-            float e = 0.0f;
-            for (int j = 0; j < kClusterCtas; ++j) e += pe[j];
-            ear_tok[t - nclusters] = e;
-          }
+          if (live)
+            kl_tok[t] = (W / Sa) * inv_temp - ((Ma - Mb) * inv_temp + (lg2(Sa) - lg2(Sb)) * kLn2);
+          if (i > 0) ear_tok[t - nclusters] = E;
         }
       }
     }
@@ -450,9 +371,9 @@ __global__ void __launch_bounds__(kClusterThreads, 1)
         }
       }
     }
-    const float3 es = block_sum3<kClusterThreads>(e_acc[0] + e_acc[1], 0.0f, 0.0f, red);
-    if (threadIdx.x == 0) ear_part[buf] = es.x;
-    // block_sum3 ended with __syncthreads: every read of this buffer is done.
+    const float es = block_sum<kClusterThreads>(e_acc[0] + e_acc[1]);
+    if (threadIdx.x == 0) ear_part[buf] = es;
+    // block_sum ended with __syncthreads: every read of this buffer is done.
     if (threadIdx.x == 0 && !aborted && issued < nrows && issued == i + 2) {
       fence_proxy_async_smem();
       issue(issued);
@@ -463,13 +384,13 @@ __global__ void __launch_bounds__(kClusterThreads, 1)
   if (rank == 0 && threadIdx.x == 0 && nrows > 0) {
     const int buf = static_cast<int>((nrows - 1) & 1);
     float e = 0.0f;
-    for (int j = 0; j < kClusterCtas; ++j) e += cluster.map_shared_rank(ear_part, j)[buf];
+    for (int j = 0; j < CS; ++j) e += cluster.map_shared_rank(ear_part, j)[buf];
     ear_tok[cluster_id + (nrows - 1) * nclusters] = e;
   }
   // Copies issued but never consumed (only after a timeout) must land first.
   if (threadIdx.x == 0 && aborted) {
     for (int64_t i = (issued > 2 ? issued - 2 : 0); i < issued; ++i)
-      mbar_wait_bounded(&full[i & 1], static_cast<uint32_t>((i >> 1) & 1), kWaitLimitNs);
+      mbar_wait_bounded(&full[i & 1], static_cast<uint32_t>((i >> 1) & 1));
   }
   cluster.sync();  // keep shared memory alive until rank 0 has read it
 }
@@ -500,8 +421,54 @@ __global__ void __launch_bounds__(1024)
   }
 }
 
-constexpr size_t kClusterSmemExtra = 16 + 2 * sizeof(SliceStat) + 8 + sizeof(SliceStat) +
-                                     (3 * (kClusterThreads / 32) + 2) * sizeof(float) + 64;
+constexpr size_t kClusterSmemExtra = 16 + 2 * sizeof(SliceStat) + 8 + sizeof(SliceStat) + 64;
+
+// Launch the cluster kernel with CS CTAs per cluster if the GPU can keep such
+// clusters resident; returns the number of resident CTAs it would use (0 if
+// the configuration is impossible) and launches only when `launch` is set.
+template <int CS>
+int64_t cluster_launch(bool launch, const uint16_t* a, const uint16_t* b, int64_t T, int64_t V,
+                       float c, float inv_temp, float* ear_tok, float* kl_tok, uint32_t* flags,
+                       cudaStream_t stream, cudaError_t* err) {
+  const int64_t v8 = V / 8;
+  const int64_t upc = (v8 + CS - 1) / CS;
+  const size_t smem = static_cast<size_t>(4 * upc * 16) + kClusterSmemExtra;
+  if (smem > 220 * 1024) return 0;
+  if (cudaFuncSetAttribute(ear_kl_cluster_kernel<CS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  if (CS > 8 && cudaFuncSetAttribute(ear_kl_cluster_kernel<CS>,
+                                     cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kClusterThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.gridDim = dim3(CS * 32, 1, 1);
+  int max_clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&max_clusters, ear_kl_cluster_kernel<CS>, &cfg) != cudaSuccess)
+    max_clusters = 0;
+  cudaGetLastError();
+  if (max_clusters <= 0) return 0;
+  const int64_t nc = T < max_clusters ? T : max_clusters;
+  if (launch) {
+    cfg.gridDim = dim3(static_cast<unsigned>(CS * nc), 1, 1);
+    *err = cudaLaunchKernelEx(&cfg, ear_kl_cluster_kernel<CS>, a, b, T, V, static_cast<int>(upc),
+                              c, inv_temp, ear_tok, kl_tok, flags);
+  }
+  return static_cast<int64_t>(max_clusters) * CS;
+}
 
 }  // namespace
 
@@ -515,40 +482,22 @@ cudaError_t launch_ear_kl(const uint16_t* a, const uint16_t* b, int64_t T, int64
   const float c = 1.4426950408889634f * inv_temp;
   cudaError_t err = cudaSuccess;
 
-  // Single-pass cluster kernel when rows are 16-byte aligned and a slice pair
-  // (double-buffered) fits in shared memory; the row kernel otherwise.
-  const int64_t v8 = V / 8;
-  const int64_t upc = (v8 + kClusterCtas - 1) / kClusterCtas;
-  const size_t smem = static_cast<size_t>(4 * upc * 16) + kClusterSmemExtra;
+  // Single-pass cluster kernel when rows are 16-byte aligned and the slices
+  // fit in shared memory; the configuration with more resident CTAs wins
+  // (16-CTA clusters halve the slice, so two CTAs can share an SM).  The row
+  // kernel covers every other case.
   bool done = false;
-  if (V % 8 == 0 && smem <= 220 * 1024) {
-    err = cudaFuncSetAttribute(ear_kl_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
-    if (err != cudaSuccess) return err;
-    cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(kClusterThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kClusterCtas;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cfg.gridDim = dim3(kClusterCtas * 64, 1, 1);
-    int max_clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&max_clusters, ear_kl_cluster_kernel, &cfg) != cudaSuccess)
-      max_clusters = 0;
-    cudaGetLastError();
-    if (max_clusters > 0) {
-      const int64_t nc = T < max_clusters ? T : max_clusters;
-      cfg.gridDim = dim3(static_cast<unsigned>(kClusterCtas * nc), 1, 1);
-      err = cudaLaunchKernelEx(&cfg, ear_kl_cluster_kernel, a, b, T, V, static_cast<int>(upc), c,
-                               inv_temp, ear_tok, kl_tok, flags);
-      if (err != cudaSuccess) return err;
+  if (V % 8 == 0) {
+    const int64_t r16 = cluster_launch<16>(false, a, b, T, V, c, inv_temp, ear_tok, kl_tok, flags, stream, &err);
+    const int64_t r8 = cluster_launch<8>(false, a, b, T, V, c, inv_temp, ear_tok, kl_tok, flags, stream, &err);
+    if (r16 > 0 && r16 >= r8) {
+      cluster_launch<16>(true, a, b, T, V, c, inv_temp, ear_tok, kl_tok, flags, stream, &err);
+      done = true;
+    } else if (r8 > 0) {
+      cluster_launch<8>(true, a, b, T, V, c, inv_temp, ear_tok, kl_tok, flags, stream, &err);
       done = true;
     }
+    if (err != cudaSuccess) return err;
   }
   if (!done) {
     constexpr int kThreads = 1024;

@@ -34,6 +34,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include "dequant.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -41,6 +42,10 @@ namespace cg = cooperative_groups;
 
 namespace slq {
 namespace {
+
+using dq::load_unit;
+using dq::sw128_desc;
+using dq::unit_pairs;
 
 constexpr int kBM = 128;     // W rows per tile (MMA M)
 constexpr int kBK = 64;      // k per A / X stage: one 128-byte swizzle atom of bf16
@@ -50,25 +55,24 @@ constexpr int kWorkers = 8;  // dequant + accumulate warps
 constexpr int kMaxCluster = 8;
 constexpr int kWarpX = 0, kWarpMma = 1, kWarpW = 2, kWarp0 = 3;
 constexpr int kThreads = (kWarp0 + kWorkers) * 32;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 template <int B>
 constexpr int p_stage_bytes() {
   return kBM * 16 * B;
 }
 
-// Stage counts and the shared-memory budget.  Narrow tiles (BN <= 64, the
-// decode and small-batch shapes) aim for two CTAs per SM and spend what is
-// left of ~110 KB on packed-W stages, so that many bytes of weights are in
-// flight; wide tiles use one CTA per SM.
+// Stage counts and the shared-memory budget.  The decode tile (BN = 16) aims
+// for two CTAs per SM and spends what is left of 112 KB on packed-W stages;
+// wider tiles use one CTA per SM and up to 227 KB, so that many bytes of
+// weights are in flight either way.
 template <int B, int BN>
 struct Cfg {
-  static constexpr int kSX = BN == 256 ? 3 : 4;
+  static constexpr int kSX = BN == 16 ? 8 : (BN == 256 ? 3 : 4);
   static constexpr int kXStage = BN * 128;
   static constexpr int kAStage = kBM * 128;
   static constexpr int kFixed = 1024 /* alignment slack */ + kSX * kXStage + kSA * kAStage +
                                 kSRing * kBM * 3 + 512 /* barriers, TMEM address, flag */;
-  static constexpr int kBudget = BN <= 64 ? 110 * 1024 : 227 * 1024;
+  static constexpr int kBudget = BN == 16 ? 112 * 1024 : 227 * 1024;
   static constexpr int kSPRaw = (kBudget - kFixed) / p_stage_bytes<B>();
   static constexpr int kSP = kSPRaw > 8 ? 8 : (kSPRaw < 2 ? 2 : kSPRaw);
   static constexpr int kSmem = kFixed + kSP * p_stage_bytes<B>();
@@ -80,116 +84,6 @@ struct Cfg {
   static_assert(BN > 64 || kSA * kAStage >= kBM * BN * 4,
                 "A stages double as the split-K partial buffer");
 };
-
-// Physical byte offset of a logical offset inside a packed-W stage, for the
-// swizzle mode its tensor map uses (128/64/32-byte rows for b = 8/4/2).
-template <int B>
-__device__ __forceinline__ uint32_t p_swz(uint32_t off) {
-  if constexpr (B == 8) return off ^ (((off >> 7) & 7u) << 4);
-  else if constexpr (B == 4) return off ^ (((off >> 7) & 3u) << 4);
-  else if constexpr (B == 2) return off ^ (((off >> 7) & 1u) << 4);
-  else return off;
-}
-
-// b words (32 codes) of row `row`, unit u (codes [32u, 32u+32)) of a stage.
-template <int B>
-__device__ __forceinline__ void load_unit(const uint8_t* st, int row, int u, uint32_t (&w)[B]) {
-  if constexpr (B == 8) {
-    const uint32_t off = row * 128 + 32 * u;
-    const uint4 v0 = *reinterpret_cast<const uint4*>(st + p_swz<8>(off));
-    const uint4 v1 = *reinterpret_cast<const uint4*>(st + p_swz<8>(off + 16));
-    w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
-    w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
-  } else if constexpr (B == 4) {
-    const uint4 v = *reinterpret_cast<const uint4*>(st + p_swz<4>(row * 64 + 16 * u));
-    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-  } else if constexpr (B == 2) {
-    const uint2 v = *reinterpret_cast<const uint2*>(st + p_swz<2>(row * 32 + 8 * u));
-    w[0] = v.x; w[1] = v.y;
-  } else if constexpr (B == 6) {
-    const uint8_t* p = st + row * 96 + 24 * u;
-#pragma unroll
-    for (int i = 0; i < 3; ++i) {
-      const uint2 v = *reinterpret_cast<const uint2*>(p + 8 * i);
-      w[2 * i] = v.x; w[2 * i + 1] = v.y;
-    }
-  } else {
-    const uint32_t* p = reinterpret_cast<const uint32_t*>(st + row * 16 * B + 4 * B * u);
-#pragma unroll
-    for (int i = 0; i < B; ++i) w[i] = p[i];
-  }
-}
-
-template <int B>
-__device__ __forceinline__ uint32_t code_at(const uint32_t (&w)[B], int i) {
-  const int o = B * i;
-  const int wi = o >> 5;
-  const int sh = o & 31;
-  constexpr uint32_t mask = (1u << B) - 1u;
-  if (sh + B <= 32) return (w[wi] >> sh) & mask;
-  return __funnelshift_r(w[wi], w[wi + 1], sh) & mask;
-}
-
-__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
-  __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a),
-                             *reinterpret_cast<__nv_bfloat162*>(&b));
-  return *reinterpret_cast<uint32_t*>(&r);
-}
-
-// The 32 codes of a unit as 16 bf16x2 registers (q_{2p} - z, q_{2p+1} - z),
-// consecutive k, exact.  For b <= 7 each code is ORed into the mantissa of
-// bf16 128.0 and (128 + z) is subtracted in bf16; b = 8 goes through binary32
-// (2^23 + q) - (2^23 + z).  For b = 4 and b = 2 one byte is isolated with a
-// byte permute and a multiply by 0x1001 / 0x4001 places its two codes 16 bits
-// apart, so a single AND/OR forms the pair.
-template <int B>
-__device__ __forceinline__ void unit_pairs(const uint32_t (&w)[B], uint32_t z, uint32_t (&out)[16]) {
-  if constexpr (B == 8) {
-    const float zf = __uint_as_float(0x4B000000u | z);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const float lo = __uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7540 | (2 * h)));
-        const float hi = __uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7540 | (2 * h + 1)));
-        __nv_bfloat162 v = __floats2bfloat162_rn(__fsub_rn(lo, zf), __fsub_rn(hi, zf));
-        out[2 * i + h] = *reinterpret_cast<uint32_t*>(&v);
-      }
-    }
-  } else {
-    const uint32_t z2 = (0x4300u | z) * 0x00010001u;  // bf16x2 (128 + z, 128 + z)
-    if constexpr (B == 4) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t y = __byte_perm(w[i], 0u, 0x4440 | k) * 0x1001u;
-          out[4 * i + k] = bf16x2_sub((y & 0x000F000Fu) | 0x43004300u, z2);
-        }
-    } else if constexpr (B == 2) {
-#pragma unroll
-      for (int i = 0; i < 2; ++i)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t y = __byte_perm(w[i], 0u, 0x4440 | k) * 0x4001u;
-          out[8 * i + 2 * k] = bf16x2_sub((y & 0x00030003u) | 0x43004300u, z2);
-          out[8 * i + 2 * k + 1] = bf16x2_sub(((y >> 4) & 0x00030003u) | 0x43004300u, z2);
-        }
-    } else {
-#pragma unroll
-      for (int p = 0; p < 16; ++p)
-        out[p] = bf16x2_sub(code_at<B>(w, 2 * p) | (code_at<B>(w, 2 * p + 1) << 16) | 0x43004300u, z2);
-    }
-  }
-}
-
-// UMMA shared-memory descriptor: K-major, 128-byte swizzle, 8-row groups
-// 1024 bytes apart (SBO), descriptor version 1 (sm_100).
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
-         (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
-         (static_cast<uint64_t>(2) << 61);
-}
 
 // Instruction descriptor, kind::f16: bf16 A and B (K-major), fp32 D, M = 128, N = BN.
 template <int BN>
@@ -208,19 +102,23 @@ struct Bars {
   uint64_t* pf;  // P buffer filled (tcgen05.commit)
   uint64_t* pe;  // P buffer drained by the workers
   uint64_t* mma_done;
+  uint64_t* done;  // decode tile: MMAs of group g complete (ring of 4)
   uint32_t* tmem_base;
   volatile int* abort_flag;
 };
 
 // Bounded wait; on timeout raises the flag word and the CTA-wide abort flag.
+// The cycle counter and the abort flag are read only every few polls.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, const Bars& sh,
                                               uint32_t* flags) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  const long long t0 = clock64();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+#pragma unroll 1
+    for (int i = 0; i < 8; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
     if (*sh.abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (clock64() - t0 > kWaitLimitCycles) {
       *sh.abort_flag = 1;
       if (flags) atomicOr(flags, kFlagTimeout);
       return false;
@@ -231,13 +129,25 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, co
 template <int B, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmap_x,
-                      const __grid_constant__ CUtensorMap tmap_w, int M, int N, int K,
+                      const __grid_constant__ CUtensorMap tmap_w, const uint16_t* __restrict__ X,
+                      int M, int N, int K,
                       const uint16_t* __restrict__ scales, const uint8_t* __restrict__ zeros,
                       void* __restrict__ Y, int y_f32, int groups_per_slice,
                       uint32_t* __restrict__ flags) {
   using C = Cfg<B, BN>;
   constexpr int kSP = C::kSP;
-  constexpr int kCols = 2 * BN;  // two P buffers
+  // The 8 K=16 MMAs of a group go to kChains independent accumulators (MMA k
+  // into chain k mod kChains).  With the 16-wide decode tile each MMA is tiny
+  // and a single dependent chain runs at the tensor core's latency, not its
+  // throughput; four chains overlap.  Wider tiles keep one chain.
+  constexpr int kChains = BN == 16 ? 4 : 1;
+  // Decode tile: one commit per group (done[g % 4]) stands for "A stages,
+  // X stages and P buffer of group g are free / ready"; the MMA thread waits
+  // only for the second k-block of a group, which both producers publish
+  // after the first.  This keeps the single issuing thread's per-group
+  // latency (waits, commits) small next to its eight MMAs.
+  constexpr bool kDec = BN == 16;
+  constexpr int kCols = 2 * kChains * BN;  // two P buffers of kChains accumulators
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -257,7 +167,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   sh.pf = sh.p_empty + kSP;
   sh.pe = sh.pf + 2;
   sh.mma_done = sh.pe + 2;
-  sh.tmem_base = reinterpret_cast<uint32_t*>(sh.mma_done + 1);
+  sh.done = sh.mma_done + 1;
+  sh.tmem_base = reinterpret_cast<uint32_t*>(sh.done + 4);
   sh.abort_flag = reinterpret_cast<volatile int*>(sh.tmem_base + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -273,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kSX; ++i) {
-      mbar_init(&sh.x_full[i], 1);
+      mbar_init(&sh.x_full[i], BN == 16 ? 32 : 1);  // decode: one arrival per producer lane
       mbar_init(&sh.x_empty[i], 1);
     }
     for (int i = 0; i < kSA; ++i) {
@@ -289,6 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sh.pe[i], kWorkers);
     }
     mbar_init(sh.mma_done, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&sh.done[i], 1);
     *sh.abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -302,8 +214,52 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *sh.tmem_base;
 
-  if (warp == kWarpX) {
-    // ---------------- X producer ----------------
+  if (warp == kWarpX && BN == 16) {
+    // ---------------- X producer, decode tile ----------------
+    // The 16 x 64 X tile of a k-block is only a few rows of activations that
+    // every CTA reads; all 32 lanes copy it with 16-byte cp.async (rows >= M
+    // zero-filled), kXAhead k-blocks ahead, and publish a stage once its
+    // copies have landed (wait_group, then a proxy fence for tcgen05.mma).
+    constexpr int kXAhead = 4;
+    static_assert(BN != 16 || kXAhead < C::kSX, "X lookahead must leave a free stage");
+    auto copy_kblock = [&](int kb) {
+      const int s = kb % C::kSX;
+      uint8_t* dst = xbuf + s * C::kXStage;
+      const int64_t k0 = static_cast<int64_t>(2 * g_begin + kb) * kBK;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int v = lane + 32 * j;  // 16 rows x 8 chunks of 16 bytes
+        const int r = v >> 3, c = v & 7;
+        const bool in = (m0 + r) < M;
+        const uint16_t* src = in ? X + static_cast<int64_t>(m0 + r) * K + k0 + 8 * c : X;
+        cp_async_16(dst + r * 128 + ((c ^ (r & 7)) << 4), src, in ? 16u : 0u);
+      }
+    };
+    bool ok = true;
+    for (int kb = 0; kb < kXAhead && kb < KB; ++kb) {
+      copy_kblock(kb);  // the first stages are free
+      cp_async_commit();
+    }
+    for (int kb = 0; kb < KB && ok; ++kb) {
+      const int kn = kb + kXAhead;
+      if (kn < KB) {
+        bool w = true;
+        if (kn >= C::kSX) {  // the stage held k-block kn - kSX: its group's MMAs must be done
+          const int gx = (kn - C::kSX) >> 1;
+          w = wait_or_abort(&sh.done[gx & 3], (gx >> 2) & 1, sh, flags);
+        }
+        ok = __all_sync(0xffffffffu, w);
+        if (ok) copy_kblock(kn);
+      }
+      cp_async_commit();  // possibly empty: keeps one group per k-block
+      cp_async_wait<kXAhead>();  // the group of k-block kb has landed
+      fence_proxy_async_smem();
+      mbar_arrive(&sh.x_full[kb % C::kSX]);
+    }
+    cp_async_wait<0>();  // nothing in flight past this point
+    __syncwarp();
+  } else if (warp == kWarpX) {
+    // ---------------- X producer (TMA) ----------------
     if (lane == 0) {
       prefetch_tmap(&tmap_x);
       int issued = 0;
@@ -316,14 +272,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // Drain: every issued copy must land before the CTA may exit.
       for (int i = issued - C::kSX; i < issued; ++i)
-        if (i >= 0) mbar_wait_bounded(&sh.x_full[i % C::kSX], (i / C::kSX) & 1, kWaitLimitNs);
+        if (i >= 0) mbar_wait_bounded(&sh.x_full[i % C::kSX], (i / C::kSX) & 1);
     }
     __syncwarp();
   } else if (warp == kWarpW) {
     // ---------------- packed-W producer + scale / zero staging ----------------
-    // Lane l stages rows 4l..4l+3.  The scale / zero loads run kLookahead
-    // groups ahead of the stores (a register pipeline), so their DRAM latency
-    // overlaps the ring instead of stalling every group.
+    // Lane l stages rows 4l..4l+3.  Scale / zero loads are issued kLookahead
+    // groups before they are stored: the loop is unrolled by kLookahead so slot
+    // j of the register ring is only read when its load, issued kLookahead
+    // iterations earlier, has had time to land -- the DRAM latency overlaps
+    // the ring instead of stalling every group.
     if (lane == 0) prefetch_tmap(&tmap_w);
     constexpr int kLookahead = BN <= 64 ? 8 : 4;
     auto fetch = [&](int g, int q) -> uint32_t {
@@ -332,39 +290,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t gi = static_cast<int64_t>(n) * G + g_begin + g;
       return static_cast<uint32_t>(scales[gi]) | (static_cast<uint32_t>(zeros[gi]) << 16);
     };
-    uint32_t pipe[kLookahead][4];
+    uint32_t ring[kLookahead][4];
 #pragma unroll
     for (int j = 0; j < kLookahead; ++j)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) pipe[j][q] = fetch(j, q);
+      for (int q = 0; q < 4; ++q) ring[j][q] = fetch(j, q);
     int issued = 0;
-    for (int g = 0; g < ng; ++g) {
-      const int s = g % kSP;
-      const bool ok = wait_or_abort(&sh.p_empty[s], ((g / kSP) & 1) ^ 1, sh, flags);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&sh.p_full[s], p_stage_bytes<B>());
-        tma_load_2d(pbuf + s * p_stage_bytes<B>(), &tmap_w, &sh.p_full[s], (g_begin + g) * 4 * B, n0);
+    bool run = true;
+    for (int g0 = 0; g0 < ng && run; g0 += kLookahead) {
+#pragma unroll
+      for (int j = 0; j < kLookahead; ++j) {
+        const int g = g0 + j;
+        if (g >= ng || !run) break;
+        const int s = g % kSP;
+        const bool ok = wait_or_abort(&sh.p_empty[s], ((g / kSP) & 1) ^ 1, sh, flags);
+        if (!__all_sync(0xffffffffu, ok)) {
+          run = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&sh.p_full[s], p_stage_bytes<B>());
+          tma_load_2d(pbuf + s * p_stage_bytes<B>(), &tmap_w, &sh.p_full[s], (g_begin + g) * 4 * B, n0);
+        }
+        uint16_t* sr = sring + (g % kSRing) * kBM;
+        uint8_t* zr = zring + (g % kSRing) * kBM;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          sr[4 * lane + q] = static_cast<uint16_t>(ring[j][q] & 0xFFFFu);
+          zr[4 * lane + q] = static_cast<uint8_t>(ring[j][q] >> 16);
+        }
+        mbar_arrive(&sh.p_full[s]);
+        ++issued;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) ring[j][q] = fetch(g + kLookahead, q);
       }
-      uint16_t* sr = sring + (g % kSRing) * kBM;
-      uint8_t* zr = zring + (g % kSRing) * kBM;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        sr[4 * lane + q] = static_cast<uint16_t>(pipe[0][q] & 0xFFFFu);
-        zr[4 * lane + q] = static_cast<uint8_t>(pipe[0][q] >> 16);
-      }
-      mbar_arrive(&sh.p_full[s]);
-      ++issued;
-#pragma unroll
-      for (int j = 0; j < kLookahead - 1; ++j)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) pipe[j][q] = pipe[j + 1][q];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) pipe[kLookahead - 1][q] = fetch(g + kLookahead, q);
     }
     if (lane == 0)
       for (int i = issued - kSP; i < issued; ++i)
-        if (i >= 0) mbar_wait_bounded(&sh.p_full[i % kSP], (i / kSP) & 1, kWaitLimitNs);
+        if (i >= 0) mbar_wait_bounded(&sh.p_full[i % kSP], (i / kSP) & 1);
     __syncwarp();
   } else if (warp == kWarpMma) {
     // ---------------- MMA issuer: group g into P[g % 2] ----------------
@@ -376,7 +339,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = wait_or_abort(&sh.pe[buf], ((g >> 1) & 1) ^ 1, sh, flags);
         if (!ok) break;
         tc_fence_after_sync();
-        const uint32_t d = tmem + static_cast<uint32_t>(buf * BN);
+        const uint32_t d = tmem + static_cast<uint32_t>(buf * kChains * BN);
+        if constexpr (kDec) {
+          const int kb1 = 2 * g + 1;
+          ok = wait_or_abort(&sh.a_full[kb1 % kSA], (kb1 / kSA) & 1, sh, flags) &&
+               wait_or_abort(&sh.x_full[kb1 % C::kSX], (kb1 / C::kSX) & 1, sh, flags);
+          if (!ok) break;
+          tc_fence_after_sync();
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int kb = 2 * g + h;
+            const uint64_t da = sw128_desc(smem_u32(abuf + (kb % kSA) * C::kAStage));
+            const uint64_t db = sw128_desc(smem_u32(xbuf + (kb % C::kSX) * C::kXStage));
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k) {
+              const int kk = h * (kBK / 16) + k;
+              umma_bf16_ss(d + static_cast<uint32_t>((kk % kChains) * BN), da + 2 * k, db + 2 * k,
+                           idesc, kk >= kChains ? 1u : 0u);
+            }
+          }
+          umma_commit(&sh.done[g & 3]);
+          continue;
+        }
 #pragma unroll 1
         for (int h = 0; h < 2 && ok; ++h) {
           const int kb = 2 * g + h;
@@ -388,15 +372,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t da = sw128_desc(smem_u32(abuf + sa * C::kAStage));
           const uint64_t db = sw128_desc(smem_u32(xbuf + sx * C::kXStage));
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k)  // +32 bytes along K per MMA: +2 in the address field
-            umma_bf16_ss(d, da + 2 * k, db + 2 * k, idesc, (h > 0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < kBK / 16; ++k) {  // +32 bytes along K per MMA: +2 in the address field
+            const int kk = h * (kBK / 16) + k;  // MMA index within the group
+            umma_bf16_ss(d + static_cast<uint32_t>((kk % kChains) * BN), da + 2 * k, db + 2 * k,
+                         idesc, kk >= kChains ? 1u : 0u);
+          }
           umma_commit(&sh.a_empty[sa]);
           umma_commit(&sh.x_empty[sx]);
         }
         if (ok) umma_commit(&sh.pf[buf]);
       }
       umma_commit(sh.mma_done);
-      mbar_wait_bounded(sh.mma_done, 0, kWaitLimitNs);  // no MMA in flight past this point
+      mbar_wait_bounded(sh.mma_done, 0);  // no MMA in flight past this point
     }
     __syncwarp();
   } else {
@@ -415,9 +402,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (g < ng) {
         // ---- dequantize group g into A stages 2g, 2g+1 ----
         const int sp = g % kSP;
-        ok = wait_or_abort(&sh.a_empty[(2 * g) % kSA], (((2 * g) / kSA) & 1) ^ 1, sh, flags) &&
-             wait_or_abort(&sh.a_empty[(2 * g + 1) % kSA], (((2 * g + 1) / kSA) & 1) ^ 1, sh, flags) &&
-             wait_or_abort(&sh.p_full[sp], (g / kSP) & 1, sh, flags);
+        if constexpr (kDec) {  // A stages of group g - 2 are free once its MMAs are done
+          ok = (g < 2 || wait_or_abort(&sh.done[(g - 2) & 3], ((g - 2) >> 2) & 1, sh, flags)) &&
+               wait_or_abort(&sh.p_full[sp], (g / kSP) & 1, sh, flags);
+        } else {
+          ok = wait_or_abort(&sh.a_empty[(2 * g) % kSA], (((2 * g) / kSA) & 1) ^ 1, sh, flags) &&
+               wait_or_abort(&sh.a_empty[(2 * g + 1) % kSA], (((2 * g + 1) / kSA) & 1) ^ 1, sh, flags) &&
+               wait_or_abort(&sh.p_full[sp], (g / kSP) & 1, sh, flags);
+        }
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         const uint8_t* pst = pbuf + sp * p_stage_bytes<B>();
@@ -450,13 +442,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---- fold P_{g-1} into the accumulators: acc += s[n, g-1] * P ----
         const int j = g - 1;
         const int buf = j & 1;
-        ok = __all_sync(0xffffffffu, wait_or_abort(&sh.pf[buf], (j >> 1) & 1, sh, flags));
+        if constexpr (kDec)
+          ok = __all_sync(0xffffffffu, wait_or_abort(&sh.done[j & 3], (j >> 2) & 1, sh, flags));
+        else
+          ok = __all_sync(0xffffffffu, wait_or_abort(&sh.pf[buf], (j >> 1) & 1, sh, flags));
         if (!ok) break;
         tc_fence_after_sync();
         const float s =
             __half2float(__ushort_as_half(sring[(j % kSRing) * kBM + 32 * q + lane]));
         const uint32_t base = tmem + (static_cast<uint32_t>(32 * q) << 16) +
-                              static_cast<uint32_t>(buf * BN + hcol * kHalf);
+                              static_cast<uint32_t>(buf * kChains * BN + hcol * kHalf);
         if constexpr (kHalf % 16 == 0) {
 #pragma unroll
           for (int c = 0; c < kHalf / 16; ++c) {
@@ -467,11 +462,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 16; ++i) acc[16 * c + i] = fmaf(s, __uint_as_float(r[i]), acc[16 * c + i]);
           }
         } else {
-          uint32_t r[8];
-          tmem_ld_32x32b_x8(base, r);
+          // Decode tile: sum the kChains partial accumulators in a fixed order.
+          uint32_t r[kChains][8];
+#pragma unroll
+          for (int c = 0; c < kChains; ++c) tmem_ld_32x32b_x8(base + static_cast<uint32_t>(c * BN), r[c]);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] = fmaf(s, __uint_as_float(r[i]), acc[i]);
+          for (int i = 0; i < 8; ++i) {
+            float v = __uint_as_float(r[0][i]);
+#pragma unroll
+            for (int c = 1; c < kChains; ++c) v += __uint_as_float(r[c][i]);
+            acc[i] = fmaf(s, v, acc[i]);
+          }
         }
         tc_fence_before_sync();
         __syncwarp();
@@ -559,29 +561,19 @@ cudaError_t launch_cfg(const uint16_t* X, int M, int N, int K, const uint32_t* p
   cudaError_t e = cudaFuncSetAttribute(gemm_tiled_kernel<B, BN>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
+  // Ask for the largest shared-memory carveout so that two decode CTAs fit
+  // on an SM (the default carveout may hold only one).
+  e = cudaFuncSetAttribute(gemm_tiled_kernel<B, BN>,
+                           cudaFuncAttributePreferredSharedMemoryCarveout,
+                           static_cast<int>(cudaSharedmemCarveoutMaxShared));
+  if (e != cudaSuccess) return e;
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int G = K / kGroup;
   const int row_blocks = (N + kBM - 1) / kBM;
   const int col_blocks = (M + BN - 1) / BN;
-  // Narrow tiles: split K over a cluster so that the CTAs fill the resident
-  // slots (two per SM) in one wave without spilling into a second one; each
-  // slice keeps at least four groups.
-  int C_split = 1;
-  if (BN <= 64) {
-    const int tiles = row_blocks * col_blocks;
-    C_split = (2 * sms) / tiles;
-    if (C_split > kMaxCluster) C_split = kMaxCluster;
-    if (C_split > G / 4) C_split = G / 4;
-    if (C_split < 1) C_split = 1;
-  }
-  const int per_slice = (G + C_split - 1) / C_split;
-  C_split = (G + per_slice - 1) / per_slice;  // no empty slices
-
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(row_blocks), static_cast<unsigned>(col_blocks),
-                     static_cast<unsigned>(C_split));
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = stream;
@@ -589,10 +581,40 @@ cudaError_t launch_cfg(const uint16_t* X, int M, int N, int K, const uint32_t* p
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = static_cast<unsigned>(C_split);
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemm_tiled_kernel<B, BN>, tx, tw, M, N, K, scales, zeros, Y,
+
+  // Narrow tiles: split K over a cluster of C CTAs, with the largest C (at
+  // most 8, each slice keeping at least four groups) for which every cluster
+  // of the launch is resident at once -- the occupancy API decides, since
+  // cluster placement, not only shared memory, limits residency.
+  int C_split = 1;
+  if (BN <= 64) {
+    static int max_active[kMaxCluster + 1] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};
+    const int tiles = row_blocks * col_blocks;
+    for (int c = kMaxCluster; c >= 2; --c) {
+      if (c > G / 4) continue;
+      if (max_active[c] < 0) {
+        attr[0].val.clusterDim.z = static_cast<unsigned>(c);
+        cfg.gridDim = dim3(1, 1, static_cast<unsigned>(c));
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, gemm_tiled_kernel<B, BN>, &cfg) != cudaSuccess) n = 0;
+        cudaGetLastError();
+        max_active[c] = n;
+      }
+      if (tiles <= max_active[c]) {
+        C_split = c;
+        break;
+      }
+    }
+  }
+  const int per_slice = (G + C_split - 1) / C_split;
+  C_split = (G + per_slice - 1) / per_slice;  // no empty slices
+
+  cfg.gridDim = dim3(static_cast<unsigned>(row_blocks), static_cast<unsigned>(col_blocks),
+                     static_cast<unsigned>(C_split));
+  attr[0].val.clusterDim.z = static_cast<unsigned>(C_split);
+  return cudaLaunchKernelEx(&cfg, gemm_tiled_kernel<B, BN>, tx, tw, X, M, N, K, scales, zeros, Y,
                             y_f32 ? 1 : 0, per_slice, flags);
 }
 

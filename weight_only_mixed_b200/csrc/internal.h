@@ -24,6 +24,13 @@ bool encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const voi
                           uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
                           uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
+// Decode dequantize-GEMM (M <= 16): dequant to TMEM + tcgen05.mma with the
+// weights as the TMEM operand, split-K over a cluster.
+cudaError_t launch_gemm_decode(const uint16_t* X, int64_t M, int64_t N, int64_t K, int bits,
+                               const uint32_t* packed, const uint16_t* scales,
+                               const uint8_t* zeros, void* Y, bool y_f32, uint32_t* flags,
+                               cudaStream_t stream);
+
 // Dequantize-GEMM on tcgen05 (TMA + dequant to shared memory + tcgen05.mma
 // with TMEM accumulators).  decode = true selects the 16-wide activation tile
 // with split-K over a cluster (M <= 16); otherwise the tile width follows M.

@@ -8,16 +8,18 @@
 // the plain round-to-nearest baseline the reddit excerpt names (RTN).
 //
 // Kernel shape: one warp per 128-weight group.  Lane l holds weights
-// [4l, 4l+4) (one 8-byte load), the min/max are warp-shuffle reductions, every
+// [4l, 4l+4) (one 8-byte load), the min/max are warp reductions, every
 // lane derives the same fp16 scale and zero point, and the 4 codes of a lane
 // form a 4b-bit chunk at stream bit 4b*l.  Lane j < 4b then gathers word j of
 // the group from the (at most five) lanes whose chunks overlap it and stores
 // it, so a group's 4b words leave as one coalesced store.  HBM-bound: 2 bytes
 // read and b/8 + 3/128 bytes written per weight.
 //
-// Bit-exactness with the binary32 definition: IEEE division (__fdiv_rn),
-// rintf (round half to even), __float2half_rn (round to nearest even, fp16
-// subnormals kept), no flush-to-zero and no FMA contraction on these paths.
+// Bit-exactness with the binary32 definition: IEEE division (__fdiv_rn) for
+// the scale and zero point and wherever the reciprocal product could round
+// differently (rne_quotient), rintf (round half to even), __float2half_rn
+// (round to nearest even, fp16 subnormals kept), no flush-to-zero and no FMA
+// contraction on these paths.
 #include <cuda_fp16.h>
 
 #include "internal.h"
@@ -33,6 +35,32 @@ constexpr int kUnroll = 4;  // groups per warp per iteration (loads in flight)
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
+// Warp-wide float min / max in one instruction (sm_100a redux.sync); a NaN
+// input is ignored, as with fminf / fmaxf.
+__device__ __forceinline__ float warp_min(float v) {
+  float r;
+  asm volatile("redux.sync.min.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+__device__ __forceinline__ float warp_max(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+
+// rne(fl32(w / s)) for the encode.  With r = RN(1/s), t = RN(w r) differs from
+// the IEEE quotient fl32(w / s) by at most 1.5 * 2^-23 * |t| (< 1.9e-4 for
+// |t| < 1024), so the two round to the same integer unless t lies within that
+// distance of a half-integer; those rare elements (exact ties among them) take
+// the IEEE division.  Beyond |t| = 1024 the code clamps to an end of the grid
+// (|z| <= 255) whichever way the quotient rounds.
+__device__ __forceinline__ float rne_quotient(float w, float s, float r) {
+  const float t = __fmul_rn(w, r);
+  float k = rintf(t);
+  if (fabsf(t) < 1024.0f && fabsf(fabsf(t - k) - 0.5f) < 2.5e-4f) k = rintf(__fdiv_rn(w, s));
+  return k;
+}
+
 template <int B>
 __device__ __forceinline__ void encode_group(uint2 raw, int64_t grp, int lane,
                                              uint32_t* __restrict__ packed,
@@ -45,13 +73,8 @@ __device__ __forceinline__ void encode_group(uint2 raw, int64_t grp, int lane,
   const bool any_nonfinite = __any_sync(kFull, nonfinite);
 
   // Group statistics: min and max (exact in binary32).
-  float mn = fminf(fminf(w[0], w[1]), fminf(w[2], w[3]));
-  float mx = fmaxf(fmaxf(w[0], w[1]), fmaxf(w[2], w[3]));
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    mn = fminf(mn, __shfl_xor_sync(kFull, mn, off));
-    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
-  }
+  const float mn = warp_min(fminf(fminf(w[0], w[1]), fminf(w[2], w[3])));
+  const float mx = warp_max(fmaxf(fmaxf(w[0], w[1]), fmaxf(w[2], w[3])));
 
   // A constant group is widened to include 0.
   float lo = mn, hi = mx;
@@ -79,10 +102,11 @@ __device__ __forceinline__ void encode_group(uint2 raw, int64_t grp, int lane,
   const float s = __half2float(__ushort_as_half(s16));
   const float zf = fminf(fmaxf(rintf(__fdiv_rn(-lo, s)), 0.0f), maxq);
 
+  const float r = __frcp_rn(s);
   uint32_t chunk = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float v = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(w[i], s)), zf), 0.0f), maxq);
+    const float v = fminf(fmaxf(__fadd_rn(rne_quotient(w[i], s, r), zf), 0.0f), maxq);
     chunk |= static_cast<uint32_t>(v) << (B * i);
   }
 

@@ -163,8 +163,9 @@ slq_status slq_gemm_ex(const void* X_bf16, int64_t M, int64_t N, int64_t K, int 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const uint16_t* X = static_cast<const uint16_t*>(X_bf16);
   const uint16_t* sc = static_cast<const uint16_t*>(scales_f16);
-  return from_cuda(slq::launch_gemm_tiled(X, M, N, K, bits, packed, sc, zeros, Y, f32,
-                                          path == SLQ_GEMM_DECODE, flags, s));
+  if (path == SLQ_GEMM_DECODE)
+    return from_cuda(slq::launch_gemm_decode(X, M, N, K, bits, packed, sc, zeros, Y, f32, flags, s));
+  return from_cuda(slq::launch_gemm_tiled(X, M, N, K, bits, packed, sc, zeros, Y, f32, false, flags, s));
 }
 
 slq_status slq_gemm(const void* X_bf16, int64_t M, int64_t N, int64_t K, int bits,
