@@ -46,7 +46,7 @@ _PATHS = {"auto": SLQ_GEMM_AUTO, "decode": SLQ_GEMM_DECODE, "tiled": SLQ_GEMM_TI
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m weight_only_mixed_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python weight_only_mixed_b200/build.py` "
         "(nvcc, sm_100a).  There is no fallback implementation.")
 
 _lib = ctypes.CDLL(LIB_PATH)

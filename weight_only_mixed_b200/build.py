@@ -1,6 +1,6 @@
 """Build libslq.so (sm_100a) in-tree with nvcc.
 
-    python -m weight_only_mixed_b200.build [--force]
+    python weight_only_mixed_b200/build.py [--force] [-v]
 
 Every translation unit under csrc/ is compiled for sm_100a only
 (-gencode arch=compute_100a,code=sm_100a) and linked into one shared library
