@@ -352,7 +352,7 @@ def run_slq(args, rank, world, local_rank):
             },
             "roofline": {
                 "bound": "hbm",
-                "kernel": "gemm_tiled_kernel<b, BN=16> (TMA + dequant to smem + tcgen05.mma/TMEM, split-K cluster; M<=16)",
+                "kernel": "gemm_decode_kernel<b> (TMA-staged packed W dequantized into TMEM, tcgen05.mma with the TMEM A operand, persistent stream-K over one CTA per SM; M<=16)",
                 "achieved": round(achieved, 1),
                 "peak": hbm_peak,
                 "unit": "GB/s",
@@ -421,6 +421,8 @@ def other_rows(args, slq, synth, torch, dev, stream, hbm_peak, tc_peak, rank):
                 slq.gemm(Xs, qws[it[0] % nrot], out=Ys, stream=stream)
                 it[0] += 1
 
+            slq.gemm(Xs, qws[0], out=Ys, stream=stream)  # sizes the workspace before capture
+            stream.synchronize()
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 for r in range(nrot):

@@ -54,14 +54,16 @@ enum {
   SLQ_FLAG_TIMEOUT = 4u         /* a bounded on-chip wait gave up; outputs are unspecified */
 };
 
-/* GEMM kernel configuration for slq_gemm_ex.  Every configuration runs the
- * same sm_100a kernel: TMA-staged packed weights, dequantized to exact bf16
- * (q - z) in shared memory, tcgen05.mma into TMEM per 128-wide group, and the
- * fp16 group scale applied to the fp32 group product. */
+/* GEMM kernel choice for slq_gemm_ex.  Both kernels dequantize the weights
+ * to exact bf16 (q - z), multiply on the tcgen05 tensor cores with fp32
+ * accumulation in TMEM, one product per 128-wide group, and apply the fp16
+ * group scale to that fp32 product. */
 typedef enum {
   SLQ_GEMM_AUTO = 0,   /* DECODE for M <= 16, TILED above */
-  SLQ_GEMM_DECODE = 1, /* 128 x 16 output tiles, K split over a thread-block cluster (M <= 16) */
-  SLQ_GEMM_TILED = 2   /* 128 x {64, 128, 256} output tiles sized to M (any M >= 1) */
+  SLQ_GEMM_DECODE = 1, /* M <= 16: weights dequantized into TMEM, one persistent CTA per SM,
+                          the row tiles x groups split evenly over the CTAs (needs a workspace) */
+  SLQ_GEMM_TILED = 2   /* any M >= 1: 128 x {64, 128, 256} output tiles, weights dequantized
+                          into shared memory, K split over a thread-block cluster for M <= 64 */
 } slq_gemm_path;
 
 /* Group size along K, fixed by the format ("asymmetric INT, group size 128",
@@ -85,6 +87,19 @@ size_t slq_packed_words(int64_t N, int64_t K, int bits);
 /* Which kernel slq_gemm would run for these sizes (SLQ_GEMM_DECODE or
  * SLQ_GEMM_TILED).  Host-only; launches nothing. */
 slq_gemm_path slq_gemm_select(int64_t M, int64_t N, int64_t K, int bits);
+
+/* Bytes of device workspace slq_gemm needs for Y[M, N] = X[M, K] W[N, K]^T
+ * on the CURRENT device (the decode kernel splits the layer over that
+ * device's SMs); 0 when the call needs none (M > 16, or every row tile falls
+ * in one CTA).  Returns 0 for invalid arguments.
+ *
+ * Workspace rules: device memory owned by the caller, 256-byte aligned, not
+ * overlapping any other argument, ALL ZERO before its first use.  Every call
+ * that completes without SLQ_FLAG_TIMEOUT leaves it all zero again, so one
+ * buffer serves any number of calls issued one after another on a stream;
+ * calls that may run at the same time need separate buffers.  After a call
+ * that raised SLQ_FLAG_TIMEOUT the caller must zero it again. */
+size_t slq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits);
 
 /*
  * slq_quantize -- round-to-nearest asymmetric INT-`bits` encode of W, group
@@ -131,22 +146,28 @@ slq_status slq_quantize(const void *W_bf16, int64_t N, int64_t K, int bits,
  * bits, packed, scales_f16, zeros   as written by slq_quantize.
  * Y           [M, N] of y_dtype, device, written.  With SLQ_DTYPE_BF16 each
  *             element is the round-to-nearest-even bf16 of the fp32 value the
- *             same kernel writes with SLQ_DTYPE_F32 (the reduction order does
- *             not depend on the output type; no atomics).
+ *             same kernel writes with SLQ_DTYPE_F32: the order of every sum is
+ *             fixed by the sizes and the device, never by timing, so repeated
+ *             calls give identical bits.
+ * workspace, workspace_bytes   at least slq_gemm_workspace_bytes(M, N, K,
+ *             bits) bytes under the workspace rules above; may be NULL / 0
+ *             when that is 0.  SLQ_ERR_INVALID_ARGUMENT if too small.
  * flags       device uint32 or NULL; SLQ_FLAG_TIMEOUT.
  */
 slq_status slq_gemm(const void *X_bf16, int64_t M, int64_t N, int64_t K,
                     int bits, const uint32_t *packed, const void *scales_f16,
                     const uint8_t *zeros, void *Y, slq_dtype y_dtype,
-                    uint32_t *flags, void *stream);
+                    void *workspace, size_t workspace_bytes, uint32_t *flags,
+                    void *stream);
 
-/* slq_gemm with an explicit kernel choice (SLQ_GEMM_DECODE needs M <= 16).
- * Same arguments and results otherwise. */
+/* slq_gemm with an explicit kernel choice (SLQ_GEMM_DECODE needs M <= 16;
+ * the workspace requirement is that of the chosen kernel: none for
+ * SLQ_GEMM_TILED).  Same arguments and results otherwise. */
 slq_status slq_gemm_ex(const void *X_bf16, int64_t M, int64_t N, int64_t K,
                        int bits, const uint32_t *packed,
                        const void *scales_f16, const uint8_t *zeros, void *Y,
-                       slq_dtype y_dtype, slq_gemm_path path, uint32_t *flags,
-                       void *stream);
+                       slq_dtype y_dtype, slq_gemm_path path, void *workspace,
+                       size_t workspace_bytes, uint32_t *flags, void *stream);
 
 /*
  * slq_ear_kl -- per-token Expected Acceptance Rate and KL divergence between

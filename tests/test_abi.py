@@ -79,9 +79,14 @@ def test_quantize_validation():
     assert _q(N=0) == slq.SLQ_OK  # empty: nothing to do, nothing launched
 
 
+WS = FAKE + (6 << 24)
+
+
 def _g(M=4, N=8, K=256, bits=4, X=FAKE, packed=FAKE + (1 << 24), scales=FAKE + (2 << 24),
-       zeros=FAKE + (3 << 24), Y=FAKE + (4 << 24), dtype=0, path=0, flags=None):
-    return L.slq_gemm_ex(X, M, N, K, bits, packed, scales, zeros, Y, dtype, path, flags, None)
+       zeros=FAKE + (3 << 24), Y=FAKE + (4 << 24), dtype=0, path=0, ws=WS, ws_bytes=1 << 24,
+       flags=None):
+    return L.slq_gemm_ex(X, M, N, K, bits, packed, scales, zeros, Y, dtype, path, ws, ws_bytes,
+                         flags, None)
 
 
 def test_gemm_validation():
@@ -93,6 +98,24 @@ def test_gemm_validation():
     for kw in bad:
         assert _g(**kw) == slq.SLQ_ERR_INVALID_ARGUMENT, kw
     assert _g(M=0) == slq.SLQ_OK and _g(N=0) == slq.SLQ_OK
+
+
+def test_gemm_workspace_rules():
+    # A layer whose row tiles are split over several CTAs needs a workspace.
+    M, N, K, b = 4, 4096, 4096, 4
+    need = slq.gemm_workspace_bytes(M, N, K, b)
+    assert need > 0
+    assert slq.gemm_workspace_bytes(17, N, K, b) == 0  # tiled kernel: none
+    assert slq.gemm_workspace_bytes(4, N, 100, b) == 0  # invalid K
+    kw = dict(M=M, N=N, K=K, bits=b)
+    big = dict(packed=FAKE + (1 << 28), scales=FAKE + (2 << 28), zeros=FAKE + (3 << 28),
+               Y=FAKE + (4 << 28), ws=FAKE + (5 << 28))
+    for bad in [dict(ws=None), dict(ws_bytes=need - 1), dict(ws=FAKE + (5 << 28) + 16),
+                dict(ws=FAKE + 256)]:  # misaligned, overlapping X
+        args = {**kw, **big, "ws_bytes": need, **bad}
+        assert _g(**args) == slq.SLQ_ERR_INVALID_ARGUMENT, bad
+    # The tiled kernel ignores the workspace.
+    assert _g(**{**kw, **big, "ws": None, "ws_bytes": 0, "path": 2}) != slq.SLQ_ERR_INVALID_ARGUMENT
 
 
 def _e(T=4, V=1000, tau=1.0, a=FAKE, b=FAKE + (1 << 24), ear=FAKE + (2 << 24),

@@ -182,3 +182,36 @@ def test_sweep_8192_prefill(bits):
 @pytest.mark.parametrize("N,K,bits", sorted(set(LLAMA_70B)))
 def test_llama_70b_block_prefill(N, K, bits):
     _sampled_prefill_check(N, K, bits, Ms=[64, 2048])
+
+
+# ---------------------------------------------------------------------------
+# Decode kernel: stream-K split, workspace contract, determinism
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("N,K,bits,M", [(4096, 4096, 4, 16), (1024, 4096, 8, 1), (300, 128 * 37, 3, 5),
+                                        (12288, 4096, 2, 4)])
+def test_decode_workspace_left_zero_and_repeatable(N, K, bits, M):
+    W = synth.weights_torch(N, K, seed=321 + bits)
+    qw = slq.quantize(W, bits)
+    X = synth.activations_torch(M, K, seed=322)
+    need = slq.gemm_workspace_bytes(M, N, K, bits)
+    ws = torch.zeros(max(need, 256) + 4096, dtype=torch.uint8, device="cuda")
+    y1 = slq.gemm(X, qw, out_dtype=torch.float32, path="decode", workspace=ws)
+    torch.cuda.synchronize()
+    # Partial sums may stay behind; the per-tile counters must be zero again.
+    ncnt = (N + 127) // 128
+    assert int(ws[:4 * ncnt].count_nonzero()) == 0, "tile counters not reset"
+    for _ in range(3):
+        y2 = slq.gemm(X, qw, out_dtype=torch.float32, path="decode", workspace=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(y1.view(torch.int32), y2.view(torch.int32))
+    assert int(ws[:4 * ncnt].count_nonzero()) == 0
+
+
+def test_decode_flags_stay_clear():
+    N, K, bits = 2048, 8192, 5
+    qw = slq.quantize(synth.weights_torch(N, K, seed=5), bits)
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for M in (1, 7, 16):
+        slq.gemm(synth.activations_torch(M, K, seed=M), qw, flags=flags)
+    torch.cuda.synchronize()
+    assert int(flags.item()) == 0

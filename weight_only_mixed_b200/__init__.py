@@ -65,9 +65,12 @@ _lib.slq_gemm_select.argtypes = [_I64, _I64, _I64, _I]
 _lib.slq_gemm_select.restype = _I
 _lib.slq_quantize.argtypes = [_P, _I64, _I64, _I, _P, _P, _P, _P, _P]
 _lib.slq_quantize.restype = _I
-_lib.slq_gemm.argtypes = [_P, _I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _P, _P]
+_SZ = ctypes.c_size_t
+_lib.slq_gemm_workspace_bytes.argtypes = [_I64, _I64, _I64, _I]
+_lib.slq_gemm_workspace_bytes.restype = _SZ
+_lib.slq_gemm.argtypes = [_P, _I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _P, _SZ, _P, _P]
 _lib.slq_gemm.restype = _I
-_lib.slq_gemm_ex.argtypes = [_P, _I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _I, _P, _P]
+_lib.slq_gemm_ex.argtypes = [_P, _I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _I, _P, _SZ, _P, _P]
 _lib.slq_gemm_ex.restype = _I
 _lib.slq_ear_kl.argtypes = [_P, _P, _I64, _I64, ctypes.c_float, _P, _P, _P, _P, _P, _P]
 _lib.slq_ear_kl.restype = _I
@@ -106,6 +109,31 @@ def packed_words(N: int, K: int, bits: int) -> int:
 
 def gemm_select(M: int, N: int, K: int, bits: int) -> str:
     return {SLQ_GEMM_DECODE: "decode", SLQ_GEMM_TILED: "tiled"}[_lib.slq_gemm_select(M, N, K, bits)]
+
+
+def gemm_workspace_bytes(M: int, N: int, K: int, bits: int) -> int:
+    """Device workspace bytes slq_gemm needs on the current device."""
+    return int(_lib.slq_gemm_workspace_bytes(M, N, K, bits))
+
+
+# One zero-filled workspace per (device, stream), grown on demand.  The
+# library leaves it zero after every call, and calls on one stream never
+# overlap, so a stream can reuse its buffer.  Growing it allocates, so a
+# CUDA-graph capture should be preceded by an eager call of the largest size.
+_workspaces: dict = {}
+
+
+def workspace_for(nbytes: int, stream=None):
+    import torch
+    if nbytes == 0:
+        return None
+    s = stream if stream is not None else torch.cuda.current_stream()
+    key = (s.device.index, int(s.cuda_stream))
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=s.device)
+        _workspaces[key] = ws
+    return ws
 
 
 def _check(status: int, what: str):
@@ -161,8 +189,11 @@ def quantize(W, bits: int, out: QuantizedWeight | None = None, flags=None, strea
 
 
 def gemm(X, qw: QuantizedWeight, out_dtype=None, path: str = "auto", out=None, flags=None,
-         stream=None):
-    """Y = X W^T for bf16 X [M, K] and a packed layer; Y is bf16 or fp32 [M, N]."""
+         stream=None, workspace=None):
+    """Y = X W^T for bf16 X [M, K] and a packed layer; Y is bf16 or fp32 [M, N].
+
+    `workspace` (a zero-filled uint8 CUDA tensor) defaults to the stream's
+    cached buffer."""
     import torch
     out_dtype = out_dtype or torch.bfloat16
     assert X.dtype == torch.bfloat16 and X.is_cuda and X.is_contiguous() and X.dim() == 2
@@ -170,9 +201,14 @@ def gemm(X, qw: QuantizedWeight, out_dtype=None, path: str = "auto", out=None, f
     assert K == qw.K
     y = out if out is not None else torch.empty((M, qw.N), dtype=out_dtype, device=X.device)
     dt = SLQ_DTYPE_F32 if y.dtype == torch.float32 else SLQ_DTYPE_BF16
+    need = 0
+    if path != "tiled":
+        need = gemm_workspace_bytes(M, qw.N, K, qw.bits) if path == "auto" or M <= 16 else 0
+    ws = workspace if workspace is not None else workspace_for(need, stream)
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check(_lib.slq_gemm_ex(_ptr(X), M, qw.N, K, qw.bits, _ptr(qw.packed), _ptr(qw.scales),
-                            _ptr(qw.zeros), _ptr(y), dt, _PATHS[path], _ptr(flags),
-                            _stream_ptr(stream)), "slq_gemm")
+                            _ptr(qw.zeros), _ptr(y), dt, _PATHS[path], _ptr(ws), ws_bytes,
+                            _ptr(flags), _stream_ptr(stream)), "slq_gemm")
     return y
 
 

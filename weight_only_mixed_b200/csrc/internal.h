@@ -25,11 +25,17 @@ bool encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const voi
                           uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
 // Decode dequantize-GEMM (M <= 16): dequant to TMEM + tcgen05.mma with the
-// weights as the TMEM operand, split-K over a cluster.
+// weights as the TMEM operand, persistent stream-K over one CTA per SM.
+// `workspace` holds the split tiles' counters and partial sums
+// (gemm_decode_workspace_bytes; zero-filled counters on entry and exit).
 cudaError_t launch_gemm_decode(const uint16_t* X, int64_t M, int64_t N, int64_t K, int bits,
                                const uint32_t* packed, const uint16_t* scales,
-                               const uint8_t* zeros, void* Y, bool y_f32, uint32_t* flags,
-                               cudaStream_t stream);
+                               const uint8_t* zeros, void* Y, bool y_f32, void* workspace,
+                               uint32_t* flags, cudaStream_t stream);
+
+// Workspace bytes of launch_gemm_decode for an [N, K] layer on the current
+// device (0 when no row tile is split).
+size_t gemm_decode_workspace_bytes(int64_t N, int64_t K);
 
 // Dequantize-GEMM on tcgen05 (TMA + dequant to shared memory + tcgen05.mma
 // with TMEM accumulators).  decode = true selects the 16-wide activation tile

@@ -74,9 +74,18 @@ bool valid_k(int64_t K) { return K >= slq::kGroup && K % slq::kGroup == 0 && K <
 
 bool product_ok(int64_t a, int64_t b) { return a == 0 || b <= kMaxElems / a; }
 
+// Workspace of the kernel `path` selects (only the decode kernel uses one).
+size_t workspace_needed(int64_t M, int64_t N, int64_t K, slq_gemm_path path) {
+  if (path == SLQ_GEMM_AUTO) path = M <= 16 ? SLQ_GEMM_DECODE : SLQ_GEMM_TILED;
+  return (path == SLQ_GEMM_DECODE && M >= 1 && M <= 16 && N >= 1)
+             ? slq::gemm_decode_workspace_bytes(N, K)
+             : 0;
+}
+
 slq_status validate_gemm(const void* X, int64_t M, int64_t N, int64_t K, int bits,
                          const uint32_t* packed, const void* scales, const uint8_t* zeros,
-                         void* Y, slq_dtype y_dtype, uint32_t* flags) {
+                         void* Y, slq_dtype y_dtype, slq_gemm_path path, void* workspace,
+                         size_t workspace_bytes, uint32_t* flags) {
   if (M < 0 || N < 0 || M > kMaxDim || N > kMaxDim || !valid_k(K) || !valid_bits(bits))
     return SLQ_ERR_INVALID_ARGUMENT;
   if (!product_ok(M, K) || !product_ok(N, K) || !product_ok(M, N)) return SLQ_ERR_INVALID_ARGUMENT;
@@ -86,12 +95,16 @@ slq_status validate_gemm(const void* X, int64_t M, int64_t N, int64_t K, int bit
   if (!aligned(X, 16) || !aligned(packed, 16) || !aligned(Y, 16) || !aligned(scales, 2) ||
       (flags && !aligned(flags, 4)))
     return SLQ_ERR_INVALID_ARGUMENT;
+  const size_t need = workspace_needed(M, N, K, path);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256)))
+    return SLQ_ERR_INVALID_ARGUMENT;
   const int64_t G = K / slq::kGroup;
   const Range ins[4] = {range_of(X, M * K * 2), range_of(packed, N * K * bits / 8),
                         range_of(scales, N * G * 2), range_of(zeros, N * G)};
-  const Range outs[2] = {range_of(Y, M * N * (y_dtype == SLQ_DTYPE_F32 ? 4 : 2)),
-                         range_of(flags, flags ? 4 : 0)};
-  if (!disjoint(outs, 2, ins, 4)) return SLQ_ERR_INVALID_ARGUMENT;
+  const Range outs[3] = {range_of(Y, M * N * (y_dtype == SLQ_DTYPE_F32 ? 4 : 2)),
+                         range_of(flags, flags ? 4 : 0),
+                         range_of(workspace, static_cast<int64_t>(need))};
+  if (!disjoint(outs, 3, ins, 4)) return SLQ_ERR_INVALID_ARGUMENT;
   return SLQ_OK;
 }
 
@@ -145,16 +158,23 @@ slq_status slq_quantize(const void* W_bf16, int64_t N, int64_t K, int bits, uint
                                         static_cast<cudaStream_t>(stream)));
 }
 
+size_t slq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits) {
+  if (M < 0 || N < 0 || M > kMaxDim || N > kMaxDim || !valid_k(K) || !valid_bits(bits) ||
+      !product_ok(N, K))
+    return 0;
+  return workspace_needed(M, N, K, SLQ_GEMM_AUTO);
+}
+
 slq_status slq_gemm_ex(const void* X_bf16, int64_t M, int64_t N, int64_t K, int bits,
                        const uint32_t* packed, const void* scales_f16, const uint8_t* zeros,
-                       void* Y, slq_dtype y_dtype, slq_gemm_path path, uint32_t* flags,
-                       void* stream) {
-  const slq_status v =
-      validate_gemm(X_bf16, M, N, K, bits, packed, scales_f16, zeros, Y, y_dtype, flags);
-  if (v != SLQ_OK) return v;
+                       void* Y, slq_dtype y_dtype, slq_gemm_path path, void* workspace,
+                       size_t workspace_bytes, uint32_t* flags, void* stream) {
   if (path != SLQ_GEMM_AUTO && path != SLQ_GEMM_DECODE && path != SLQ_GEMM_TILED)
     return SLQ_ERR_INVALID_ARGUMENT;
   if (path == SLQ_GEMM_DECODE && M > 16) return SLQ_ERR_INVALID_ARGUMENT;
+  const slq_status v = validate_gemm(X_bf16, M, N, K, bits, packed, scales_f16, zeros, Y, y_dtype,
+                                     path, workspace, workspace_bytes, flags);
+  if (v != SLQ_OK) return v;
   if (M == 0 || N == 0) return SLQ_OK;
   const slq_status dev = check_device();
   if (dev != SLQ_OK) return dev;
@@ -164,15 +184,17 @@ slq_status slq_gemm_ex(const void* X_bf16, int64_t M, int64_t N, int64_t K, int 
   const uint16_t* X = static_cast<const uint16_t*>(X_bf16);
   const uint16_t* sc = static_cast<const uint16_t*>(scales_f16);
   if (path == SLQ_GEMM_DECODE)
-    return from_cuda(slq::launch_gemm_decode(X, M, N, K, bits, packed, sc, zeros, Y, f32, flags, s));
+    return from_cuda(
+        slq::launch_gemm_decode(X, M, N, K, bits, packed, sc, zeros, Y, f32, workspace, flags, s));
   return from_cuda(slq::launch_gemm_tiled(X, M, N, K, bits, packed, sc, zeros, Y, f32, false, flags, s));
 }
 
 slq_status slq_gemm(const void* X_bf16, int64_t M, int64_t N, int64_t K, int bits,
                     const uint32_t* packed, const void* scales_f16, const uint8_t* zeros, void* Y,
-                    slq_dtype y_dtype, uint32_t* flags, void* stream) {
+                    slq_dtype y_dtype, void* workspace, size_t workspace_bytes, uint32_t* flags,
+                    void* stream) {
   return slq_gemm_ex(X_bf16, M, N, K, bits, packed, scales_f16, zeros, Y, y_dtype, SLQ_GEMM_AUTO,
-                     flags, stream);
+                     workspace, workspace_bytes, flags, stream);
 }
 
 slq_status slq_ear_kl(const void* logits_p_bf16, const void* logits_q_bf16, int64_t T, int64_t V,
