@@ -215,3 +215,20 @@ def test_decode_flags_stay_clear():
         slq.gemm(synth.activations_torch(M, K, seed=M), qw, flags=flags)
     torch.cuda.synchronize()
     assert int(flags.item()) == 0
+
+
+@pytest.mark.parametrize("N,K,bits,M", [(8192, 8192, 5, 16), (4096, 12288, 4, 16), (8192, 8192, 8, 9)])
+def test_decode_repeated_calls_identical(N, K, bits, M):
+    """Twenty calls on one layer give identical bits, each on a freshly zeroed
+    workspace and on a reused one (catches races on the staged buffers and on
+    the cross-CTA partial sums)."""
+    qw = slq.quantize(synth.weights_torch(N, K, seed=900 + bits), bits)
+    X = synth.activations_torch(M, K, seed=901)
+    need = slq.gemm_workspace_bytes(M, N, K, bits)
+    ref = slq.gemm(X, qw, out_dtype=torch.float32, path="decode")
+    reused = torch.zeros(max(need, 256), dtype=torch.uint8, device="cuda")
+    for i in range(20):
+        ws = torch.zeros(max(need, 256), dtype=torch.uint8, device="cuda") if i % 2 else reused
+        y = slq.gemm(X, qw, out_dtype=torch.float32, path="decode", workspace=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int32), ref.view(torch.int32)), i

@@ -35,7 +35,7 @@ cudaError_t launch_gemm_decode(const uint16_t* X, int64_t M, int64_t N, int64_t 
 
 // Workspace bytes of launch_gemm_decode for an [N, K] layer on the current
 // device (0 when no row tile is split).
-size_t gemm_decode_workspace_bytes(int64_t N, int64_t K);
+size_t gemm_decode_workspace_bytes(int64_t N, int64_t K, int bits);
 
 // Dequantize-GEMM on tcgen05 (TMA + dequant to shared memory + tcgen05.mma
 // with TMEM accumulators).  decode = true selects the 16-wide activation tile

@@ -75,10 +75,10 @@ bool valid_k(int64_t K) { return K >= slq::kGroup && K % slq::kGroup == 0 && K <
 bool product_ok(int64_t a, int64_t b) { return a == 0 || b <= kMaxElems / a; }
 
 // Workspace of the kernel `path` selects (only the decode kernel uses one).
-size_t workspace_needed(int64_t M, int64_t N, int64_t K, slq_gemm_path path) {
+size_t workspace_needed(int64_t M, int64_t N, int64_t K, int bits, slq_gemm_path path) {
   if (path == SLQ_GEMM_AUTO) path = M <= 16 ? SLQ_GEMM_DECODE : SLQ_GEMM_TILED;
   return (path == SLQ_GEMM_DECODE && M >= 1 && M <= 16 && N >= 1)
-             ? slq::gemm_decode_workspace_bytes(N, K)
+             ? slq::gemm_decode_workspace_bytes(N, K, bits)
              : 0;
 }
 
@@ -95,7 +95,7 @@ slq_status validate_gemm(const void* X, int64_t M, int64_t N, int64_t K, int bit
   if (!aligned(X, 16) || !aligned(packed, 16) || !aligned(Y, 16) || !aligned(scales, 2) ||
       (flags && !aligned(flags, 4)))
     return SLQ_ERR_INVALID_ARGUMENT;
-  const size_t need = workspace_needed(M, N, K, path);
+  const size_t need = workspace_needed(M, N, K, bits, path);
   if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256)))
     return SLQ_ERR_INVALID_ARGUMENT;
   const int64_t G = K / slq::kGroup;
@@ -162,7 +162,7 @@ size_t slq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits) {
   if (M < 0 || N < 0 || M > kMaxDim || N > kMaxDim || !valid_k(K) || !valid_bits(bits) ||
       !product_ok(N, K))
     return 0;
-  return workspace_needed(M, N, K, SLQ_GEMM_AUTO);
+  return workspace_needed(M, N, K, bits, SLQ_GEMM_AUTO);
 }
 
 slq_status slq_gemm_ex(const void* X_bf16, int64_t M, int64_t N, int64_t K, int bits,
