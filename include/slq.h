@@ -94,11 +94,14 @@ slq_gemm_path slq_gemm_select(int64_t M, int64_t N, int64_t K, int bits);
  * in one CTA).  Returns 0 for invalid arguments.
  *
  * Workspace rules: device memory owned by the caller, 256-byte aligned, not
- * overlapping any other argument, ALL ZERO before its first use.  Every call
- * that completes without SLQ_FLAG_TIMEOUT leaves it all zero again, so one
- * buffer serves any number of calls issued one after another on a stream;
- * calls that may run at the same time need separate buffers.  After a call
- * that raised SLQ_FLAG_TIMEOUT the caller must zero it again. */
+ * overlapping any other argument.  Its first 64 KiB hold per-row-tile
+ * counters that must be ALL ZERO before its first use; every call that
+ * completes without SLQ_FLAG_TIMEOUT leaves them zero again (the rest is
+ * scratch), so one buffer serves any number of calls -- of any layer sizes --
+ * issued one after another on a stream.  Calls that may run at the same time
+ * need separate buffers.  After a call that raised SLQ_FLAG_TIMEOUT the caller
+ * must zero the first 64 KiB again.  The decode kernel takes N up to
+ * 16384 * 128 = 2097152 (SLQ_ERR_INVALID_ARGUMENT above). */
 size_t slq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits);
 
 /*

@@ -232,3 +232,21 @@ def test_decode_repeated_calls_identical(N, K, bits, M):
         y = slq.gemm(X, qw, out_dtype=torch.float32, path="decode", workspace=ws)
         torch.cuda.synchronize()
         assert torch.equal(y.view(torch.int32), ref.view(torch.int32)), i
+
+
+def test_decode_workspace_reused_across_layer_sizes():
+    """One workspace serves layers of different N and K in any order: a
+    layer's partial sums never land on another layer's tile counters."""
+    layers = [(2048, 8192, 5, 7), (12288, 4096, 4, 1), (1024, 8192, 8, 16), (28672, 1024, 6, 3),
+              (4096, 4096, 2, 16)]
+    need = max(slq.gemm_workspace_bytes(M, N, K, b) for N, K, b, M in layers)
+    shared = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for rep in range(2):
+        for i, (N, K, b, M) in enumerate(layers):
+            qw = slq.quantize(synth.weights_torch(N, K, seed=77 + i), b)
+            X = synth.activations_torch(M, K, seed=78 + i)
+            fresh = torch.zeros(need, dtype=torch.uint8, device="cuda")
+            y_ref = slq.gemm(X, qw, out_dtype=torch.float32, path="decode", workspace=fresh)
+            y = slq.gemm(X, qw, out_dtype=torch.float32, path="decode", workspace=shared)
+            torch.cuda.synchronize()
+            assert torch.equal(y.view(torch.int32), y_ref.view(torch.int32)), (rep, N, K, b, M)

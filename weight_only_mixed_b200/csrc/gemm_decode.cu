@@ -74,6 +74,12 @@ constexpr int kSX = 6;                 // activation fragment stages (one group 
 constexpr int kXFrag = 8 * 32 * 8;     // one n8 tile of a group: 8 k-steps x 32 lanes x 8 B
 constexpr int kLook = 4;               // scale / zero loads in flight (groups)
 constexpr int kMaxPending = 4;         // shared tiles per CTA (at most 2 occur)
+// Workspace layout: tile counters in a fixed region at the front, partial sums
+// after it.  The counter region is the same for every layer, so partial sums
+// of one layer can never land on another layer's counters when callers reuse
+// one workspace for layers of different sizes.
+constexpr size_t kCounterBytes = size_t{64} << 10;
+constexpr int64_t kMaxRowTiles = kCounterBytes / sizeof(int);
 
 template <int B>
 constexpr int p_stage_bytes() {
@@ -564,10 +570,8 @@ cudaError_t launch_cfg(const uint16_t* X, int M, int N, int K, const uint32_t* p
     attr_set = true;
   }
   const Split sp = make_split(N, K, GS, resident_ctas());
-  const int64_t rbs = (N + kRows - 1) / kRows;
   int* counters = static_cast<int*>(workspace);
-  float* partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                             align256(static_cast<size_t>(rbs) * sizeof(int)));
+  float* partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes);
   gemm_decode_kernel<B, NT, GS><<<sp.nctas, kThreads, C::kSmem, stream>>>(
       tw, X, M, N, K, scales, zeros, Y, y_f32 ? 1 : 0, sp, counters, partials, flags);
   return cudaGetLastError();
@@ -597,9 +601,10 @@ size_t gemm_decode_workspace_bytes(int64_t N, int64_t K, int bits) {
   const Split sp = make_split(N, K, groups_per_chunk(K, bits), resident_ctas());
   const int64_t rbs = (N + kRows - 1) / kRows;
   if (sp.s_max <= 1) return 0;
-  return align256(static_cast<size_t>(rbs) * sizeof(int)) +
-         static_cast<size_t>(rbs) * sp.s_max * kMaxM * kRows * sizeof(float);
+  return kCounterBytes + static_cast<size_t>(rbs) * sp.s_max * kMaxM * kRows * sizeof(float);
 }
+
+int64_t gemm_decode_max_n() { return kMaxRowTiles * kRows; }
 
 cudaError_t launch_gemm_decode(const uint16_t* X, int64_t M, int64_t N, int64_t K, int bits,
                                const uint32_t* packed, const uint16_t* scales,

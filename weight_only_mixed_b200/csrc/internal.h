@@ -37,6 +37,10 @@ cudaError_t launch_gemm_decode(const uint16_t* X, int64_t M, int64_t N, int64_t 
 // device (0 when no row tile is split).
 size_t gemm_decode_workspace_bytes(int64_t N, int64_t K, int bits);
 
+// Largest N the decode kernel accepts (the fixed tile-counter region).
+int64_t gemm_decode_max_n();
+
+
 // Dequantize-GEMM on tcgen05 (TMA + dequant to shared memory + tcgen05.mma
 // with TMEM accumulators).  decode = true selects the 16-wide activation tile
 // with split-K over a cluster (M <= 16); otherwise the tile width follows M.

@@ -95,6 +95,8 @@ slq_status validate_gemm(const void* X, int64_t M, int64_t N, int64_t K, int bit
   if (!aligned(X, 16) || !aligned(packed, 16) || !aligned(Y, 16) || !aligned(scales, 2) ||
       (flags && !aligned(flags, 4)))
     return SLQ_ERR_INVALID_ARGUMENT;
+  if (path != SLQ_GEMM_TILED && M <= 16 && N > slq::gemm_decode_max_n())
+    return SLQ_ERR_INVALID_ARGUMENT;
   const size_t need = workspace_needed(M, N, K, bits, path);
   if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256)))
     return SLQ_ERR_INVALID_ARGUMENT;
