@@ -173,6 +173,41 @@ slq_status slq_gemm_ex(const void *X_bf16, int64_t M, int64_t N, int64_t K,
                        size_t workspace_bytes, uint32_t *flags, void *stream);
 
 /*
+ * slq_gemm_decode_static -- slq_gemm for decode batches (M <= 16) that
+ * allocates nothing and takes no workspace.
+ *
+ * The pages have no counterpart to this call; it exists for callers that
+ * cannot obtain device memory for the workspace slq_gemm needs: a plugin run
+ * inside a host engine that owns every device allocation and hands it only
+ * the layer's tensors, or a decode loop that must not call cudaMalloc
+ * (which may synchronize the device) once it is running.
+ *
+ * The decode kernel's split-K partial sums and tile counters live in a fixed
+ * array of SLQ_DECODE_STATIC_SCRATCH_BYTES bytes inside the library, one per
+ * device that loads it, held until the process exits.  Each call clears the
+ * counters (an asynchronous memset on `stream`) and then runs the same kernel
+ * as slq_gemm_ex(..., SLQ_GEMM_DECODE, ...), with the same results.
+ *
+ * Arguments, layouts and results are those of slq_gemm, without workspace.
+ *   M            0..16; larger M gives SLQ_ERR_INVALID_ARGUMENT.
+ *   Layers whose decode workspace (slq_gemm_workspace_bytes) exceeds
+ *   SLQ_DECODE_STATIC_SCRATCH_BYTES give SLQ_ERR_INVALID_ARGUMENT.
+ *
+ * Every call shares the one array of its device: calls that may run at the
+ * same time on the GPU (different streams, or several host threads) race on
+ * it and give wrong results; issue them one after another on one stream.
+ * The first call on a device looks up the array's device address (with that
+ * device current); make that first call before any stream capture.
+ */
+#define SLQ_DECODE_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
+
+slq_status slq_gemm_decode_static(const void *X_bf16, int64_t M, int64_t N,
+                                  int64_t K, int bits, const uint32_t *packed,
+                                  const void *scales_f16, const uint8_t *zeros,
+                                  void *Y, slq_dtype y_dtype, uint32_t *flags,
+                                  void *stream);
+
+/*
  * slq_ear_kl -- per-token Expected Acceptance Rate and KL divergence between
  * the next-token distributions of a reference and a quantized model.
  *

@@ -72,6 +72,8 @@ _lib.slq_gemm.argtypes = [_P, _I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _P, _SZ,
 _lib.slq_gemm.restype = _I
 _lib.slq_gemm_ex.argtypes = [_P, _I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _I, _P, _SZ, _P, _P]
 _lib.slq_gemm_ex.restype = _I
+_lib.slq_gemm_decode_static.argtypes = [_P, _I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _P, _P]
+_lib.slq_gemm_decode_static.restype = _I
 _lib.slq_ear_kl.argtypes = [_P, _P, _I64, _I64, ctypes.c_float, _P, _P, _P, _P, _P, _P]
 _lib.slq_ear_kl.restype = _I
 
@@ -209,6 +211,25 @@ def gemm(X, qw: QuantizedWeight, out_dtype=None, path: str = "auto", out=None, f
     _check(_lib.slq_gemm_ex(_ptr(X), M, qw.N, K, qw.bits, _ptr(qw.packed), _ptr(qw.scales),
                             _ptr(qw.zeros), _ptr(y), dt, _PATHS[path], _ptr(ws), ws_bytes,
                             _ptr(flags), _stream_ptr(stream)), "slq_gemm")
+    return y
+
+
+DECODE_STATIC_SCRATCH_BYTES = 8 << 20
+
+
+def gemm_decode_static(X, qw: QuantizedWeight, out_dtype=None, out=None, flags=None, stream=None):
+    """Y = X W^T for M <= 16 without a workspace (the library's fixed per-device
+    scratch array is used; calls must not overlap on the GPU)."""
+    import torch
+    out_dtype = out_dtype or torch.bfloat16
+    assert X.dtype == torch.bfloat16 and X.is_cuda and X.is_contiguous() and X.dim() == 2
+    M, K = X.shape
+    assert K == qw.K
+    y = out if out is not None else torch.empty((M, qw.N), dtype=out_dtype, device=X.device)
+    dt = SLQ_DTYPE_F32 if y.dtype == torch.float32 else SLQ_DTYPE_BF16
+    _check(_lib.slq_gemm_decode_static(_ptr(X), M, qw.N, K, qw.bits, _ptr(qw.packed),
+                                       _ptr(qw.scales), _ptr(qw.zeros), _ptr(y), dt, _ptr(flags),
+                                       _stream_ptr(stream)), "slq_gemm_decode_static")
     return y
 
 

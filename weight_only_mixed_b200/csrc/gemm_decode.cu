@@ -55,6 +55,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <mutex>
+
 #include "dequant.cuh"
 #include "internal.h"
 #include "ptx.cuh"
@@ -621,6 +623,63 @@ cudaError_t launch_gemm_decode(const uint16_t* X, int64_t M, int64_t N, int64_t 
     case 8: return launch_b<8>(X, m, n, k, packed, scales, zeros, Y, y_f32, workspace, flags, stream);
     default: return cudaErrorInvalidValue;
   }
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant: the split-K workspace lives in a fixed device
+// array of this file instead of caller memory.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t{8} << 20;  // 8 MiB per device
+
+// Zero-initialized when the library is loaded on a device; every device that
+// loads the library keeps it until the process exits.
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_ptr[kMaxDevices] = {};
+
+// The device address of g_static_scratch on the current device.  In host
+// code the array's name is only a host-side stand-in, so the address is
+// looked up (once per device, with that device current) and cached.
+cudaError_t static_scratch(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return e;
+    g_static_ptr[dev] = p;
+  }
+  *out = g_static_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+size_t gemm_decode_static_scratch_bytes() { return kStaticScratchBytes; }
+
+cudaError_t launch_gemm_decode_static(const uint16_t* X, int64_t M, int64_t N, int64_t K, int bits,
+                                      const uint32_t* packed, const uint16_t* scales,
+                                      const uint8_t* zeros, void* Y, bool y_f32, uint32_t* flags,
+                                      cudaStream_t stream) {
+  const size_t need = gemm_decode_workspace_bytes(N, K, bits);
+  if (need > kStaticScratchBytes) return cudaErrorInvalidValue;
+  void* ws = nullptr;
+  cudaError_t e = static_scratch(&ws);
+  if (e != cudaSuccess) return e;
+  if (need > 0) {
+    // The tile counters must start at zero; the partial sums need not.
+    const int64_t rbs = (N + kRows - 1) / kRows;
+    e = cudaMemsetAsync(ws, 0, static_cast<size_t>(rbs) * sizeof(int), stream);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_gemm_decode(X, M, N, K, bits, packed, scales, zeros, Y, y_f32, ws, flags, stream);
 }
 
 }  // namespace slq

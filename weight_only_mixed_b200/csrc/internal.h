@@ -40,6 +40,14 @@ size_t gemm_decode_workspace_bytes(int64_t N, int64_t K, int bits);
 // Largest N the decode kernel accepts (the fixed tile-counter region).
 int64_t gemm_decode_max_n();
 
+// launch_gemm_decode with its workspace in the library's fixed per-device
+// scratch array (gemm_decode_static_scratch_bytes bytes); cudaErrorInvalidValue
+// when the layer needs more.
+size_t gemm_decode_static_scratch_bytes();
+cudaError_t launch_gemm_decode_static(const uint16_t* X, int64_t M, int64_t N, int64_t K, int bits,
+                                      const uint32_t* packed, const uint16_t* scales,
+                                      const uint8_t* zeros, void* Y, bool y_f32, uint32_t* flags,
+                                      cudaStream_t stream);
 
 // Dequantize-GEMM on tcgen05 (TMA + dequant to shared memory + tcgen05.mma
 // with TMEM accumulators).  decode = true selects the 16-wide activation tile

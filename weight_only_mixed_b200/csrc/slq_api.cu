@@ -199,6 +199,26 @@ slq_status slq_gemm(const void* X_bf16, int64_t M, int64_t N, int64_t K, int bit
                      workspace, workspace_bytes, flags, stream);
 }
 
+slq_status slq_gemm_decode_static(const void* X_bf16, int64_t M, int64_t N, int64_t K, int bits,
+                                  const uint32_t* packed, const void* scales_f16,
+                                  const uint8_t* zeros, void* Y, slq_dtype y_dtype,
+                                  uint32_t* flags, void* stream) {
+  if (M > 16 || N > slq::gemm_decode_max_n()) return SLQ_ERR_INVALID_ARGUMENT;
+  // Validated as a call without a workspace; the size limit is checked below.
+  const slq_status v = validate_gemm(X_bf16, M, N, K, bits, packed, scales_f16, zeros, Y, y_dtype,
+                                     SLQ_GEMM_TILED, nullptr, 0, flags);
+  if (v != SLQ_OK) return v;
+  if (M == 0 || N == 0) return SLQ_OK;
+  if (slq::gemm_decode_workspace_bytes(N, K, bits) > slq::gemm_decode_static_scratch_bytes())
+    return SLQ_ERR_INVALID_ARGUMENT;
+  const slq_status dev = check_device();
+  if (dev != SLQ_OK) return dev;
+  return from_cuda(slq::launch_gemm_decode_static(
+      static_cast<const uint16_t*>(X_bf16), M, N, K, bits, packed,
+      static_cast<const uint16_t*>(scales_f16), zeros, Y, y_dtype == SLQ_DTYPE_F32, flags,
+      static_cast<cudaStream_t>(stream)));
+}
+
 slq_status slq_ear_kl(const void* logits_p_bf16, const void* logits_q_bf16, int64_t T, int64_t V,
                       float temperature, float* ear_tok, float* kl_tok, double* ear_mean,
                       double* kl_mean, uint32_t* flags, void* stream) {
