@@ -64,18 +64,17 @@
 namespace slq {
 namespace {
 
-using dq::unit_pairs;
 
-constexpr int kRows = 128;       // weight rows per tile
+constexpr int kRows = 256;       // weight rows per tile
 constexpr int kMaxM = 16;        // activation rows (two n8 mma tiles)
-constexpr int kConsumers = 8;    // consumer warps, 16 rows each
+constexpr int kConsumers = 8;    // consumer warps, 32 rows (two m16 mma tiles) each
 constexpr int kWarpW = 0, kWarpX = 1, kWarpC0 = 2;
 constexpr int kThreads = (kWarpC0 + kConsumers) * 32;
 constexpr int kCtasPerSm = 2;
 constexpr int kSX = 6;                 // activation fragment stages (one group each)
 constexpr int kXFrag = 8 * 32 * 8;     // one n8 tile of a group: 8 k-steps x 32 lanes x 8 B
-constexpr int kLook = 4;               // scale / zero loads in flight (groups)
 constexpr int kMaxPending = 4;         // shared tiles per CTA (at most 2 occur)
+constexpr int kMinChunksPerCta = 2;  // fewer CTAs rather than one-chunk slivers
 // Workspace layout: tile counters in a fixed region at the front, partial sums
 // after it.  The counter region is the same for every layer, so partial sums
 // of one layer can never land on another layer's counters when callers reuse
@@ -108,13 +107,14 @@ template <int B, int NT, int GS>
 struct Cfg {
   static constexpr int kXStage = NT * kXFrag;
   static constexpr int kStage = GS * p_stage_bytes<B>();
+  static constexpr int kSZStage = kRows * 12;  // per row: GS fp16 scales (8 B) + GS zeros (4 B)
   static constexpr int kFixed = 1024 /* alignment slack */ + kSX * kXStage +
                                 1024 /* barriers, pending list */;
   static constexpr int kBudget = 227 * 1024 / kCtasPerSm - 1024 /* static + reserved */;
-  static constexpr int kSPRaw = (kBudget - kFixed) / kStage;
+  static constexpr int kSPRaw = (kBudget - kFixed) / (kStage + kSZStage);
   static constexpr int kSP = kSPRaw > 16 ? 16 : kSPRaw;
-  static constexpr int kSmem = kFixed + kSP * kStage;
-  static_assert(kSPRaw >= 3, "shared memory budget");
+  static constexpr int kSmem = kFixed + kSP * (kStage + kSZStage);
+  static_assert(kSPRaw >= 2, "shared memory budget");
 };
 
 // The b words (32 codes) of unit t of group gs of row `row` in a chunk stage
@@ -194,6 +194,51 @@ __device__ __forceinline__ uint2 lds_v2(const void* p) {
   return r;
 }
 
+// Pair p (0..15) of a thread's unit as exact bf16 (q - z, q' - z) for the
+// consecutive codes 2p, 2p + 1; pair p feeds k-step p / 2 (even p: mma k 2t,
+// 2t+1; odd p: 2t+8, 2t+9).  z2 is bf16x2 (128 + z, 128 + z) for b <= 7, zf
+// the binary32 2^23 + z for b = 8.  For b = 4 (b = 2) a byte with the pair
+// (two pairs) is isolated with a byte permute and a multiply by 0x1001
+// (0x4001) places its codes 16 bits apart, so one LOP3 forms the pair.
+template <int B>
+__device__ __forceinline__ uint32_t pair_of(const uint32_t (&w)[B], uint32_t z2, float zf, int p) {
+  if constexpr (B == 4) {
+    const uint32_t y = __byte_perm(w[p >> 2], 0u, 0x4440 | (p & 3)) * 0x1001u;
+    return dq::bf16x2_sub((y & 0x000F000Fu) | 0x43004300u, z2);
+  } else if constexpr (B == 2) {
+    const uint32_t y = __byte_perm(w[p >> 3], 0u, 0x4440 | ((p >> 1) & 3)) * 0x4001u;
+    return dq::bf16x2_sub(((y >> (4 * (p & 1))) & 0x00030003u) | 0x43004300u, z2);
+  } else if constexpr (B == 8) {
+    const uint32_t word = w[p >> 1];
+    const int h = p & 1;
+    const float lo = __uint_as_float(__byte_perm(word, 0x4B000000u, 0x7540 | (2 * h)));
+    const float hi = __uint_as_float(__byte_perm(word, 0x4B000000u, 0x7540 | (2 * h + 1)));
+    __nv_bfloat162 v = __floats2bfloat162_rn(__fsub_rn(lo, zf), __fsub_rn(hi, zf));
+    return *reinterpret_cast<uint32_t*>(&v);
+  } else {
+    return dq::bf16x2_sub(dq::code_at<B>(w, 2 * p) | (dq::code_at<B>(w, 2 * p + 1) << 16) | 0x43004300u,
+                          z2);
+  }
+}
+
+// GS consecutive fp16 scales / uint8 zeros of one row (aligned: G % GS == 0).
+template <int GS>
+__device__ __forceinline__ uint2 ld_scales(const uint16_t* p) {
+  if constexpr (GS == 4) return ld_ro_v2(p);
+  else if constexpr (GS == 2) return make_uint2(ld_ro_u32(p), 0u);
+  else return make_uint2(static_cast<uint32_t>(*p), 0u);
+}
+template <int GS>
+__device__ __forceinline__ uint32_t ld_zeros(const uint8_t* p) {
+  if constexpr (GS == 4) return ld_ro_u32(p);
+  else if constexpr (GS == 2) return static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(p));
+  else return static_cast<uint32_t>(*p);
+}
+__device__ __forceinline__ float scale_at(uint2 v, int gs) {
+  const uint32_t w = gs < 2 ? v.x : v.y;
+  return __half2float(__ushort_as_half(static_cast<uint16_t>(w >> (16 * (gs & 1)))));
+}
+
 // Stream-K geometry shared by every CTA of a launch.
 struct Split {
   int G;        // chunks per row tile (groups / GS)
@@ -232,7 +277,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   uint8_t* pbuf = smem;                  // [kSP][128 rows][16 B GS bytes], TMA layout
   uint8_t* xbuf = pbuf + kSP * kStage;   // [kSX][NT][8 k-steps][32 lanes][8 B]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(xbuf + kSX * C::kXStage);
+  uint8_t* szbuf = xbuf + kSX * C::kXStage;  // [kSP][kRows] uint2 scales, then [kSP][kRows] u32 zeros
+  uint2* sc_st = reinterpret_cast<uint2*>(szbuf);
+  uint32_t* zc_st = reinterpret_cast<uint32_t*>(szbuf + kSP * kRows * 8);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(szbuf + kSP * C::kSZStage);
   Bars sh;
   sh.p_full = bars;
   sh.p_empty = sh.p_full + kSP;
@@ -271,128 +319,188 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     *sh.npending = 0;
     fence_mbarrier_init();
   }
+  // Launched as a programmatic dependent of the previous kernel on the stream:
+  // everything above overlapped its tail.  Before waiting for it, the first
+  // chunks of packed weights are prefetched into L2 (a prefetch cannot make
+  // a later read stale: L2 is where writes land); no global memory is read
+  // into the SM or written before the previous kernel has completed.
+  if (warp == kWarpW && lane == 0) {
+    int rb = rb0, gc = gk0 / GS;
+    for (int ci = 0; ci < nc && ci < kSP; ++ci) {
+      tma_prefetch_l2_2d(&tmap_w, gc * 4 * B * GS, rb * kRows);
+      if (++gc == Gc) {
+        gc = 0;
+        ++rb;
+      }
+    }
+  }
+  grid_dependency_wait();
   __syncthreads();
 
   if (warp == kWarpW) {
-    // ---------------- packed-W producer (TMA) ----------------
-    if (lane == 0) {
-      prefetch_tmap(&tmap_w);
-      int rb = rb0, gc = gk0 / GS;
-      int issued = 0;
-      for (int ci = 0; ci < nc; ++ci) {
-        const int s = ci % kSP;
-        if (!wait_or_abort(&sh.p_empty[s], ((ci / kSP) & 1) ^ 1, sh, flags)) break;
-        mbar_arrive_expect_tx(&sh.p_full[s], kStage);
-        tma_load_2d(pbuf + s * kStage, &tmap_w, &sh.p_full[s], gc * 4 * B * GS, rb * kRows);
-        ++issued;
-        if (++gc == Gc) {
-          gc = 0;
-          ++rb;
+    // ---------------- packed-W producer (TMA) + scale / zero staging ----------------
+    // Lane 0 issues the chunk's TMA; every lane stages the GS scales and GS
+    // zeros of rows 8l..8l+7 of the chunk into the stage's slot (one vector
+    // load per row, loaded one chunk ahead; rows past N and chunks past the
+    // range read clamped, valid addresses).  The stage is published by one
+    // arrival after the stores, with the TMA bytes on the same phase.
+    if (lane == 0) prefetch_tmap(&tmap_w);
+    int rb = rb0, gc = gk0 / GS;
+    int frb = rb0, fgc = gc;
+    // Two chunks of scales / zeros in flight (ring slot = chunk parity, so
+    // the loop is unrolled by two to keep the slot a compile-time index).
+    uint2 ns[2][8];
+    uint32_t nz[2][8];
+    auto sz_fetch = [&](uint2 (&ds)[8], uint32_t (&dz)[8]) {
+      const int rbc = min(frb, rbs - 1) * kRows;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int64_t gi = static_cast<int64_t>(min(rbc + 8 * lane + i, N - 1)) * G + fgc * GS;
+        ds[i] = ld_scales<GS>(scales + gi);
+        dz[i] = ld_zeros<GS>(zeros + gi);
+      }
+      if (++fgc == Gc) {
+        fgc = 0;
+        ++frb;
+      }
+    };
+    sz_fetch(ns[0], nz[0]);
+    sz_fetch(ns[1], nz[1]);
+    int issued = 0;
+    bool run = true;
+    for (int c0 = 0; c0 < nc && run; c0 += 2) {
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        const int ci = c0 + jj;
+        if (ci < nc && run) {
+          const int s = ci % kSP;
+          if (__all_sync(0xffffffffu, wait_or_abort(&sh.p_empty[s], ((ci / kSP) & 1) ^ 1, sh, flags))) {
+            if (lane == 0) {
+              mbar_expect_tx(&sh.p_full[s], kStage);
+              tma_load_2d(pbuf + s * kStage, &tmap_w, &sh.p_full[s], gc * 4 * B * GS, rb * kRows);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              sc_st[s * kRows + 8 * lane + i] = ns[jj][i];
+              zc_st[s * kRows + 8 * lane + i] = nz[jj][i];
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.p_full[s]);
+            sz_fetch(ns[jj], nz[jj]);  // chunk ci + 2
+            ++issued;
+            if (++gc == Gc) {
+              gc = 0;
+              ++rb;
+            }
+          } else {
+            run = false;
+          }
         }
       }
-      for (int i = issued - kSP; i < issued; ++i)  // every issued copy lands before exit
-        if (i >= 0) mbar_wait_bounded(&sh.p_full[i % kSP], (i / kSP) & 1);
     }
+    grid_launch_dependents();
+    if (lane == 0)  // every issued copy lands before exit
+      for (int i = issued - kSP; i < issued; ++i)
+        if (i >= 0) mbar_wait_bounded(&sh.p_full[i % kSP], (i / kSP) & 1);
     __syncwarp();
   } else if (warp == kWarpX) {
-    // ---------------- activation fragments (cp.async, rows >= M zero) ----------------
-    // Slot (nt, j, lane) holds X[m][k0 + 32t + 4j .. + 3], m = 8nt + lane / 4,
-    // t = lane % 4: the B fragment of k-step j for activation rows 8nt..8nt+7.
-    const int t = lane & 3;
+    // ---------------- activation fragments (rows >= M are zero) ----------------
+    // Fragment slot (nt, j, l), m = 8nt + l / 4, t = l % 4, holds
+    // X[m][k0 + 32t + 4j .. + 3]: the B fragment of k-step j for activation
+    // rows 8nt..8nt+7.  One instruction copies one activation row of the group
+    // (256 contiguous bytes): lane L takes bytes [8L, 8L + 8), i.e. t = L / 8,
+    // j = L % 8.  Rows >= M are not copied -- they only reach output columns
+    // >= M, which are never stored.  Each lane's arrival fires when its copies
+    // have landed, so this warp never waits for data, only for free stages.
     int gk = gk0;
+    const int jl = lane & 7, tl = lane >> 3;
     for (int g = 0; g < ng; ++g, gk = (gk + 1 == G) ? 0 : gk + 1) {
       const int s = g % kSX;
       if (!__all_sync(0xffffffffu,
                       wait_or_abort(&sh.x_empty[s], ((g / kSX) & 1) ^ 1, sh, flags)))
         break;
-      uint8_t* dst = xbuf + s * C::kXStage + lane * 8;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int m = 8 * nt + (lane >> 2);
-        const bool in = m < M;
-        const uint16_t* src = X + static_cast<int64_t>(in ? m : 0) * K + gk * kGroup + 32 * t;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) cp_async_8(dst + (nt * 8 + j) * 256, src + 4 * j, in ? 8u : 0u);
+      uint8_t* stage = xbuf + s * C::kXStage;
+      const uint16_t* src = X + gk * kGroup + 4 * lane;
+      for (int m = 0; m < M; ++m) {
+        const int nt = m >> 3, n = m & 7;
+        cp_async_8(stage + (nt * 8 + jl) * 256 + (4 * n + tl) * 8, src + static_cast<int64_t>(m) * K, 8u);
       }
       cp_async_mbar_arrive(&sh.x_full[s]);
     }
+    grid_launch_dependents();
     cp_async_wait<0>();  // nothing in flight past this point
     __syncwarp();
   } else {
-    // ---------------- consumers: rows 16c + lane / 4 and + 8 of the tile ----------------
+    // ---------------- consumers: rows 32c + lane / 4 + {0, 8, 16, 24} of the tile ----------------
+    // Rows 0, 1 of the thread form the m16 tile "A" of the warp, rows 2, 3
+    // tile "B"; both share each activation fragment.
     const int c = warp - kWarpC0;
     const int t = lane & 3;
-    const int r0 = 16 * c + (lane >> 2), r1 = r0 + 8;
+    int rr[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) rr[i] = 32 * c + (lane >> 2) + 8 * i;
     const bool leader = threadIdx.x == kWarpC0 * 32;
-    float acc[NT][4];
+    float acc[2][NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int h = 0; h < 2; ++h)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[nt][e] = 0.0f;
-
-    // Scales and zeros of both rows, kLook groups ahead.  Rows past N and
-    // groups past the range read clamped (valid, unused) addresses, so the
-    // loads are unconditional and nothing waits on them until they are used.
-    int frb = rb0, fgk = gk0;
-    auto sz_load = [&](uint32_t& s0, uint32_t& s1, uint32_t& z0, uint32_t& z1) {
-      const int rbc = min(frb, rbs - 1) * kRows;
-      const int64_t i0 = static_cast<int64_t>(min(rbc + r0, N - 1)) * G + fgk;
-      const int64_t i1 = static_cast<int64_t>(min(rbc + r1, N - 1)) * G + fgk;
-      s0 = scales[i0];
-      s1 = scales[i1];
-      z0 = zeros[i0];
-      z1 = zeros[i1];
-      if (++fgk == G) {
-        fgk = 0;
-        ++frb;
-      }
-    };
-    uint32_t rs0[kLook], rs1[kLook], rz0[kLook], rz1[kLook];
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-    for (int j = 0; j < kLook; ++j) sz_load(rs0[j], rs1[j], rz0[j], rz1[j]);
+        for (int e = 0; e < 4; ++e) acc[h][nt][e] = 0.0f;
 
     bool ok = true;
     int nseg = 0;  // shared row tiles met so far (the same count in every consumer warp)
     int rb = rb0, gk = gk0;
-    // The ring index j must stay a compile-time constant (the ring lives in
-    // registers), so the unrolled body is predicated instead of exited.
-    for (int g0 = 0; g0 < ng && ok; g0 += kLook) {
+    for (int ci = 0; ci < nc && ok; ++ci) {
+      const int sp_ = ci % kSP;
+      ok = __all_sync(0xffffffffu, wait_or_abort(&sh.p_full[sp_], (ci / kSP) & 1, sh, flags));
+      if (!ok) break;
+      // This chunk's scales and zeros of the four rows (staged with the codes).
+      uint2 cs[4];
+      uint32_t cz[4];
 #pragma unroll
-      for (int j = 0; j < kLook; ++j) {
-        const int g = g0 + j;
-        const int ci = g / GS, gs = g % GS;  // chunk, group within the chunk
-        const int sp_ = ci % kSP, sx = g % kSX;
-        if (g < ng && ok)
-          ok = __all_sync(0xffffffffu,
-                          (gs != 0 || wait_or_abort(&sh.p_full[sp_], (ci / kSP) & 1, sh, flags)) &&
-                              wait_or_abort(&sh.x_full[sx], (g / kSX) & 1, sh, flags));
-        if (g < ng && ok) {
-          // ---- codes of both rows -> exact bf16 (q - z) pairs ----
-          const uint8_t* pst = pbuf + sp_ * kStage;
-          uint32_t w0[B], w1[B];
-          load_codes<B, GS>(pst, r0, gs, t, w0);
-          load_codes<B, GS>(pst, r1, gs, t, w1);
+      for (int i = 0; i < 4; ++i) {
+        cs[i] = sc_st[sp_ * kRows + rr[i]];
+        cz[i] = zc_st[sp_ * kRows + rr[i]];
+      }
+      const uint8_t* pst = pbuf + sp_ * kStage;
+#pragma unroll
+      for (int gs = 0; gs < GS; ++gs) {
+        const int g = ci * GS + gs;
+        const int sx = g % kSX;
+        if (ok)
+          ok = __all_sync(0xffffffffu, wait_or_abort(&sh.x_full[sx], (g / kSX) & 1, sh, flags));
+        if (ok) {
+          // ---- codes of the four rows ----
+          uint32_t w[4][B];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) load_codes<B, GS>(pst, rr[i], gs, t, w[i]);
           if (gs == GS - 1) {
             // Release the stage only after every code word of this warp has
             // arrived in registers (the TMA refill may overwrite it at once),
             // ordered before the async proxy's writes.
             uint32_t dep = 0;
 #pragma unroll
-            for (int i = 0; i < B; ++i) dep ^= w0[i] ^ w1[i];
+            for (int i = 0; i < 4; ++i) {
+              dep ^= cs[i].x ^ cs[i].y ^ cz[i];
+#pragma unroll
+              for (int k = 0; k < B; ++k) dep ^= w[i][k];
+            }
             fence_proxy_async_smem();
             __syncwarp();
-            dep = __shfl_sync(0xffffffffu, dep, 0) | __any_sync(0xffffffffu, dep != 0);
+            dep = __any_sync(0xffffffffu, dep != 0);
             if (lane == 0) mbar_arrive_after(&sh.p_empty[sp_], dep);
           }
-          const float s0 = __half2float(__ushort_as_half(static_cast<uint16_t>(rs0[j])));
-          const float s1 = __half2float(__ushort_as_half(static_cast<uint16_t>(rs1[j])));
-          const uint32_t z0 = rz0[j], z1 = rz1[j];
-          sz_load(rs0[j], rs1[j], rz0[j], rz1[j]);
-          uint32_t p0[16], p1[16];
-          unit_pairs<B>(w0, z0, p0);
-          unit_pairs<B>(w1, z1, p1);
+          uint32_t z2[4];
+          float zf[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t z = (cz[i] >> (8 * gs)) & 0xFFu;
+            z2[i] = (0x4300u | z) * 0x00010001u;
+            zf[i] = __uint_as_float(0x4B000000u | z);
+          }
 
-          // ---- 8 k-steps; even and odd steps in separate accumulators ----
+          // ---- 8 k-steps x 2 m16 tiles; pairs made as they are used ----
           float d[2][NT][4];
 #pragma unroll
           for (int h = 0; h < 2; ++h)
@@ -403,11 +511,19 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           const uint8_t* xs = xbuf + sx * C::kXStage + lane * 8;
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
+            uint2 bfr[NT];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-              const uint2 bfr = lds_v2(xs + (nt * 8 + ks) * 256);
-              mma_bf16_16816(d[ks & 1][nt], p0[2 * ks], p1[2 * ks], p0[2 * ks + 1], p1[2 * ks + 1],
-                             bfr.x, bfr.y);
+            for (int nt = 0; nt < NT; ++nt) bfr[nt] = lds_v2(xs + (nt * 8 + ks) * 256);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int ra = 2 * h, rb_ = 2 * h + 1;
+              const uint32_t a0 = pair_of<B>(w[ra], z2[ra], zf[ra], 2 * ks);
+              const uint32_t a1 = pair_of<B>(w[rb_], z2[rb_], zf[rb_], 2 * ks);
+              const uint32_t a2 = pair_of<B>(w[ra], z2[ra], zf[ra], 2 * ks + 1);
+              const uint32_t a3 = pair_of<B>(w[rb_], z2[rb_], zf[rb_], 2 * ks + 1);
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+                mma_bf16_16816(d[h][nt], a0, a1, a2, a3, bfr[nt].x, bfr[nt].y);
             }
           }
           {
@@ -415,18 +531,23 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             // consumed its fragments (a dependency on all the accumulators).
             uint32_t dep = 0;
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-              dep ^= __float_as_uint(d[0][nt][0]) ^ __float_as_uint(d[1][nt][0]);
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) dep ^= __float_as_uint(d[h][nt][0]);
             __syncwarp();
             dep = __any_sync(0xffffffffu, dep != 0);
             if (lane == 0) mbar_arrive_after(&sh.x_empty[sx], dep);
           }
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            acc[nt][0] = fmaf(s0, d[0][nt][0] + d[1][nt][0], acc[nt][0]);
-            acc[nt][1] = fmaf(s0, d[0][nt][1] + d[1][nt][1], acc[nt][1]);
-            acc[nt][2] = fmaf(s1, d[0][nt][2] + d[1][nt][2], acc[nt][2]);
-            acc[nt][3] = fmaf(s1, d[0][nt][3] + d[1][nt][3], acc[nt][3]);
+          for (int h = 0; h < 2; ++h) {
+            const float sa = scale_at(cs[2 * h], gs), sb = scale_at(cs[2 * h + 1], gs);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              acc[h][nt][0] = fmaf(sa, d[h][nt][0], acc[h][nt][0]);
+              acc[h][nt][1] = fmaf(sa, d[h][nt][1], acc[h][nt][1]);
+              acc[h][nt][2] = fmaf(sb, d[h][nt][2], acc[h][nt][2]);
+              acc[h][nt][3] = fmaf(sb, d[h][nt][3], acc[h][nt][3]);
+            }
           }
 
           // ---- end of this CTA's part of a row tile: write it out ----
@@ -435,23 +556,27 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             const int ncover = last_cta(sp, rb) - c0 + 1;
             if (ncover == 1) {
 #pragma unroll
-              for (int nt = 0; nt < NT; ++nt)
+              for (int h = 0; h < 2; ++h)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const int m = 8 * nt + 2 * t + (e & 1);
-                  const int n = rb * kRows + (e < 2 ? r0 : r1);
-                  if (m < M && n < N) store_y(Y, y_f32, static_cast<int64_t>(m) * N + n, acc[nt][e]);
-                }
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    const int m = 8 * nt + 2 * t + (e & 1);
+                    const int n = rb * kRows + rr[2 * h + (e >> 1)];
+                    if (m < M && n < N) store_y(Y, y_f32, static_cast<int64_t>(m) * N + n, acc[h][nt][e]);
+                  }
             } else {
               const int slot = static_cast<int>(blockIdx.x) - c0;
               float* part = partials + (static_cast<int64_t>(rb) * sp.s_max + slot) * (kMaxM * kRows);
 #pragma unroll
-              for (int nt = 0; nt < NT; ++nt)
+              for (int h = 0; h < 2; ++h)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const int m = 8 * nt + 2 * t + (e & 1);
-                  if (m < M) part[m * kRows + (e < 2 ? r0 : r1)] = acc[nt][e];
-                }
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    const int m = 8 * nt + 2 * t + (e & 1);
+                    if (m < M) part[m * kRows + rr[2 * h + (e >> 1)]] = acc[h][nt][e];
+                  }
               // Each writer makes its partial visible at GPU scope before the
               // tile's counter can be advanced (the CTA barrier below is CTA
               // scope only).
@@ -471,9 +596,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
               ++nseg;
             }
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
+            for (int h = 0; h < 2; ++h)
 #pragma unroll
-              for (int e = 0; e < 4; ++e) acc[nt][e] = 0.0f;
+              for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[h][nt][e] = 0.0f;
           }
           if (++gk == G) {
             gk = 0;
@@ -483,22 +610,47 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       }
     }
 
+    // The next kernel on the stream may be scheduled once every CTA is here.
+    grid_launch_dependents();
     // Shared row tiles this CTA completed last: add the slots in slot order.
     if (leader) mbar_arrive(sh.end_bar);
     ok = __all_sync(0xffffffffu, ok && wait_or_abort(sh.end_bar, 0, sh, flags));
     if (ok) {
       const int np = *sh.npending;
-      const int ct = threadIdx.x - kWarpC0 * 32;  // 0 .. 32 * kConsumers - 1
+      const int ct = threadIdx.x - kWarpC0 * 32;  // 0 .. 32 * kConsumers - 1 == kRows - 1
+      static_assert(32 * kConsumers == kRows, "one reducing thread per tile row");
       for (int e = 0; e < np; ++e) {
         const Pending pe = sh.pending[e];
         if (!pe.last) continue;
         __threadfence();
-        const float* base = partials + static_cast<int64_t>(pe.rb) * sp.s_max * (kMaxM * kRows);
-        for (int idx = ct; idx < M * kRows; idx += 32 * kConsumers) {
-          float v = __ldcg(base + idx);
-          for (int cc = 1; cc < pe.ncover; ++cc) v += __ldcg(base + cc * (kMaxM * kRows) + idx);
-          const int m = idx / kRows, n = pe.rb * kRows + idx % kRows;
-          if (n < N) store_y(Y, y_f32, static_cast<int64_t>(m) * N + n, v);
+        // Thread ct owns row ct of the tile for every activation row m < M.
+        // The slots are added in slot order; the loads of four slots x all m
+        // are issued together so that the L2 latency is paid once per four
+        // slots, not once per value.
+        const float* base = partials + static_cast<int64_t>(pe.rb) * sp.s_max * (kMaxM * kRows) + ct;
+        float v[kMaxM];
+#pragma unroll
+        for (int m = 0; m < kMaxM; ++m) v[m] = m < M ? __ldcg(base + m * kRows) : 0.0f;
+        for (int c0 = 1; c0 < pe.ncover; c0 += 4) {
+          float u[4][kMaxM];
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+            for (int m = 0; m < kMaxM; ++m)
+              u[cc][m] = (c0 + cc < pe.ncover && m < M)
+                             ? __ldcg(base + (c0 + cc) * (kMaxM * kRows) + m * kRows)
+                             : 0.0f;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+            for (int m = 0; m < kMaxM; ++m)
+              if (c0 + cc < pe.ncover) v[m] += u[cc][m];
+        }
+        const int n = pe.rb * kRows + ct;
+        if (n < N) {
+#pragma unroll
+          for (int m = 0; m < kMaxM; ++m)
+            if (m < M) store_y(Y, y_f32, static_cast<int64_t>(m) * N + n, v[m]);
         }
         if (leader) counters[pe.rb] = 0;  // ready for the next call
       }
@@ -533,6 +685,7 @@ Split make_split(int64_t N, int64_t K, int gs, int ctas_max) {
   const int64_t total = rbs * sp.G;
   const int64_t ctas = total < ctas_max ? total : ctas_max;
   sp.per = static_cast<int>((total + ctas - 1) / ctas);
+  if (sp.per < kMinChunksPerCta) sp.per = kMinChunksPerCta;
   sp.nctas = static_cast<int>((total + sp.per - 1) / sp.per);
   // A row tile of G groups meets at most ceil((G - 1) / per) + 1 CTA ranges.
   int s = (sp.G - 1 + sp.per - 1) / sp.per + 1;
@@ -574,9 +727,18 @@ cudaError_t launch_cfg(const uint16_t* X, int M, int N, int K, const uint32_t* p
   const Split sp = make_split(N, K, GS, resident_ctas());
   int* counters = static_cast<int*>(workspace);
   float* partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes);
-  gemm_decode_kernel<B, NT, GS><<<sp.nctas, kThreads, C::kSmem, stream>>>(
-      tw, X, M, N, K, scales, zeros, Y, y_f32 ? 1 : 0, sp, counters, partials, flags);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(sp.nctas), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_decode_kernel<B, NT, GS>, tw, X, M, N, K, scales, zeros, Y,
+                            y_f32 ? 1 : 0, sp, counters, partials, flags);
 }
 
 template <int B>
