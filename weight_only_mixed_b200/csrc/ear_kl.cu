@@ -15,18 +15,20 @@
 // log-domain form needs no per-element logarithm and has no 0 * log 0 case.
 // Differences of two bf16 logits are exact in fp32, so every exponent argument
 // is one rounding away from exact.
-#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
 #include "internal.h"
 #include "ptx.cuh"
 
-namespace cg = cooperative_groups;
-
 namespace slq {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
+// Ring kernel shape: 16 consumer warps, two 16-byte units of each logit
+// stream per consumer thread per stage (a 32 KiB stage), six stages.
+constexpr int kEarConsumerWarps = 16;
+constexpr int kEarUnits = 2;
+constexpr int kEarStages = 6;
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -70,6 +72,147 @@ __device__ __forceinline__ void push(RowStat& st, float a, float b, float c) {
     st.b.m = b;
   }
   st.b.s += ex2((b - st.b.m) * c);
+}
+
+// ---------------------------------------------------------------------------
+// Packed binary32 pairs (sm_100 f32x2 instructions: one issue, two lanes).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t pk(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float pk_lo(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return lo;
+}
+__device__ __forceinline__ float pk_hi(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return hi;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// The two bf16 logits of one 32-bit word as a packed binary32 pair (exact).
+__device__ __forceinline__ uint64_t bf16x2_f32x2(uint32_t w) { return pk(bf16_lo(w), bf16_hi(w)); }
+__device__ __forceinline__ uint64_t ex2x2(uint64_t x) { return pk(ex2(pk_lo(x)), ex2(pk_hi(x))); }
+
+// Maximum of the bf16 logits in U 16-byte units (packed bf16 max tree).
+template <int U>
+__device__ __forceinline__ float units_max(const uint4 (&v)[U]) {
+  uint32_t m[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    uint32_t x, y;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(x) : "r"(v[u].x), "r"(v[u].y));
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(y) : "r"(v[u].z), "r"(v[u].w));
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(m[u]) : "r"(x), "r"(y));
+  }
+#pragma unroll
+  for (int w = 1; w < U; w *= 2)
+#pragma unroll
+    for (int u = 0; u + w < U; u += 2 * w) asm("max.bf16x2 %0, %1, %2;" : "=r"(m[u]) : "r"(m[u]), "r"(m[u + w]));
+  return fmaxf(bf16_lo(m[0]), bf16_hi(m[0]));
+}
+
+// Per-thread statistics of the vector path.  The sums are kept relative to
+// the offset o = -rn(k c), k = max(running max, -1e30), so each term is one
+// packed FMA (a c + o) and one exponential; the running maximum moves at most
+// once per group of units.  At the end the sums are brought to the exact
+// offset -k c by the factor 2^(k c + o), whose exponent an FMA gives exactly.
+struct VecStat {
+  float ma, ka, mb, kb;
+  uint64_t oa, ob;      // {o, o}
+  uint64_t sa, sb, w;   // packed partial sums
+};
+
+__device__ __forceinline__ VecStat vec_stat_init(float c) {
+  const float o = 1e30f * c;
+  return VecStat{-INFINITY, -1e30f, -INFINITY, -1e30f, pk(o, o), pk(o, o), 0ull, 0ull, 0ull};
+}
+
+template <int U>
+__device__ __forceinline__ void push_units(VecStat& st, const uint4 (&va)[U], const uint4 (&vb)[U],
+                                           float c) {
+  const uint64_t c2 = pk(c, c);
+  const float mA = units_max<U>(va), mB = units_max<U>(vb);
+  if (mA > st.ma) {
+    st.ma = mA;
+    st.ka = fmaxf(mA, -1e30f);
+    const float o = -(st.ka * c);
+    const float f = ex2(o - pk_lo(st.oa));
+    st.sa = mul2(st.sa, pk(f, f));
+    st.w = mul2(st.w, pk(f, f));
+    st.oa = pk(o, o);
+  }
+  if (mB > st.mb) {
+    st.mb = mB;
+    st.kb = fmaxf(mB, -1e30f);
+    const float o = -(st.kb * c);
+    const float f = ex2(o - pk_lo(st.ob));
+    st.sb = mul2(st.sb, pk(f, f));
+    st.ob = pk(o, o);
+  }
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const uint32_t wa[4] = {va[u].x, va[u].y, va[u].z, va[u].w};
+    const uint32_t wb[4] = {vb[u].x, vb[u].y, vb[u].z, vb[u].w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint64_t A = bf16x2_f32x2(wa[q]), B = bf16x2_f32x2(wb[q]);
+      const uint64_t ea = ex2x2(fma2(A, c2, st.oa));
+      st.sa = add2(st.sa, ea);
+      st.w = fma2(ea, sub2(A, B), st.w);
+      st.sb = add2(st.sb, ex2x2(fma2(B, c2, st.ob)));
+    }
+  }
+}
+
+__device__ __forceinline__ RowStat vec_stat_final(const VecStat& st, float c) {
+  const float fa = ex2(-fmaf(st.ka, c, pk_lo(st.oa)));
+  const float fb = ex2(-fmaf(st.kb, c, pk_lo(st.ob)));
+  return RowStat{{st.ma, (pk_lo(st.sa) + pk_hi(st.sa)) * fa},
+                 {st.mb, (pk_lo(st.sb) + pk_hi(st.sb)) * fb},
+                 (pk_lo(st.w) + pk_hi(st.w)) * fa};
+}
+
+// EAR terms of U units: 2^min(x_a, x_b) with x = (a - m) c - log2 S; the
+// shift by the row maximum is exact in binary32, so x takes one rounding.
+template <int U>
+__device__ __forceinline__ void ear_units(uint64_t (&acc)[2], const uint4 (&va)[U],
+                                          const uint4 (&vb)[U], uint64_t c2, uint64_t ma2,
+                                          uint64_t nla2, uint64_t mb2, uint64_t nlb2) {
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const uint32_t wa[4] = {va[u].x, va[u].y, va[u].z, va[u].w};
+    const uint32_t wb[4] = {vb[u].x, vb[u].y, vb[u].z, vb[u].w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint64_t xa = fma2(sub2(bf16x2_f32x2(wa[q]), ma2), c2, nla2);
+      const uint64_t xb = fma2(sub2(bf16x2_f32x2(wb[q]), mb2), c2, nlb2);
+      const float x0 = fminf(pk_lo(xa), pk_lo(xb)), x1 = fminf(pk_hi(xa), pk_hi(xb));
+      acc[q & 1] = add2(acc[q & 1], pk(ex2(x0), ex2(x1)));
+    }
+  }
 }
 
 __device__ __forceinline__ void merge_stat(Stat& x, float& wx, const Stat& y, float wy, float c,
@@ -146,11 +289,255 @@ __device__ float block_sum(float v) {
   return r;
 }
 
+// Row statistics plus an EAR partial, reduced together.
+struct Part {
+  RowStat st;
+  float ear;
+};
+
+__device__ __forceinline__ Part warp_reduce(Part v, float c) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    merge(v.st, shfl_xor(v.st, off), c);
+    v.ear += __shfl_xor_sync(kFull, v.ear, off);
+  }
+  return v;
+}
+
+__device__ __forceinline__ float kl_of(const RowStat& r, float inv_temp) {
+  constexpr float kLn2 = 0.693147180559945309f;
+  const float la = lg2(r.a.s), lb = lg2(r.b.s);
+  return (r.w / r.a.s) * inv_temp - ((r.a.m - r.b.m) * inv_temp + (la - lb) * kLn2);
+}
+
 // ---------------------------------------------------------------------------
-// Row-per-CTA kernel, any V: pass 1 = online statistics, pass 2 = EAR terms
-// (the second read of the row mostly hits L2).  16-byte loads when V % 8 == 0.
+// V % 8 == 0 (16-byte aligned rows): one CTA per SM walks its rows t0,
+// t0 + G, ...  A producer warp streams each row twice through a ring of
+// shared-memory stages with 1-D bulk copies -- chunks of the row for the
+// statistics pass (from HBM, kept in L2), then the same chunks again for the
+// EAR pass (from L2) -- so loads are always in flight, independent of the
+// arithmetic.  kCW consumer warps process the stages: each thread takes kU
+// 16-byte units of each logit stream per stage.  Between the passes the
+// consumer warps reduce the row statistics through shared memory; the EAR
+// sum of a row is reduced together with the statistics of the next one.
+// Every wait is bounded; a timeout raises SLQ_FLAG_TIMEOUT and the CTA stops.
 // ---------------------------------------------------------------------------
-template <int kThreads, bool kVec>
+template <int kCW, int kU>
+struct RingCfg {
+  static constexpr int kConsumers = kCW * 32;
+  static constexpr int kThreads = kConsumers + 32;
+  static constexpr int kChunk = kU * 8 * kConsumers;  // logits of one stream per stage
+  static constexpr int kStageBytes = 2 * kChunk * 2;  // a and b
+};
+
+__device__ __forceinline__ bool ring_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 8; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+template <int kCW, int kU, int kStages>
+__global__ void __launch_bounds__(RingCfg<kCW, kU>::kThreads, 1)
+    ear_kl_ring_kernel(const uint16_t* __restrict__ A, const uint16_t* __restrict__ Bq, int64_t T,
+                       int64_t V, float c, float inv_temp, float* __restrict__ ear_tok,
+                       float* __restrict__ kl_tok, uint32_t* __restrict__ flags) {
+  using Cfg = RingCfg<kCW, kU>;
+  constexpr int kChunk = Cfg::kChunk;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint16_t* stages = reinterpret_cast<uint16_t*>(smem);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * Cfg::kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* red = empty + kStages;  // [2]
+  Part* parts = reinterpret_cast<Part*>(red + 2);  // [2][kCW]
+  volatile int* abort = reinterpret_cast<volatile int*>(parts + 2 * kCW);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t G = gridDim.x;
+  const int64_t nch = (V + kChunk - 1) / kChunk;  // chunks per pass of one row
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kCW);
+    }
+    mbar_init(&red[0], kCW);
+    mbar_init(&red[1], kCW);
+    *abort = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+
+  if (warp == kCW) {
+    // Producer: one lane issues every copy, in the consumers' order.
+    if (lane != 0) return;
+    const uint64_t keep = l2_policy_evict_last();
+    const uint64_t done = l2_policy_evict_first();
+    uint32_t seq = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < T && ok; t += G) {
+      for (int pass = 0; pass < 2 && ok; ++pass) {
+        for (int64_t k = 0; k < nch; ++k, ++seq) {
+          const int s = static_cast<int>(seq % kStages);
+          if (seq >= static_cast<uint32_t>(kStages) &&
+              !ring_wait(&empty[s], ((seq / kStages) & 1u) ^ 1u, abort)) {
+            ok = false;
+            break;
+          }
+          const int64_t v0 = k * kChunk;
+          const uint32_t bytes = static_cast<uint32_t>((V - v0 < kChunk ? V - v0 : kChunk) * 2);
+          uint16_t* dst = stages + static_cast<size_t>(s) * (2 * kChunk);
+          mbar_arrive_expect_tx(&full[s], 2 * bytes);
+          bulk_load_hint(dst, A + t * V + v0, bytes, &full[s], pass ? done : keep);
+          bulk_load_hint(dst + kChunk, Bq + t * V + v0, bytes, &full[s], pass ? done : keep);
+        }
+      }
+    }
+    if (!ok) {
+      // Consumers stopped: let the copies already issued land before exit.
+      const uint32_t first = seq > static_cast<uint32_t>(kStages) ? seq - kStages : 0u;
+      for (uint32_t q = first; q < seq; ++q)
+        mbar_wait_bounded(&full[q % kStages], (q / kStages) & 1u);
+      if (flags) atomicOr(flags, kFlagTimeout);
+    }
+    return;
+  }
+
+  // Consumers.
+  const int ct = threadIdx.x;  // 0 .. kConsumers-1
+  const Part none{{{-INFINITY, 0.0f}, {-INFINITY, 0.0f}, 0.0f}, 0.0f};
+  uint32_t seq = 0, nred = 0;
+  int64_t t_prev = -1;
+  float ear_part = 0.0f;
+  // One stage: load this thread's units (all of them, or those inside a
+  // ragged last chunk), release the stage once the loads have returned, then
+  // run `f` on the loaded units.
+  auto consume = [&](int64_t k, auto&& f_full, auto&& f_one) -> bool {
+    const int s = static_cast<int>(seq % kStages);
+    if (!ring_wait(&full[s], (seq / kStages) & 1u, abort)) return false;
+    const uint16_t* a_st = stages + static_cast<size_t>(s) * (2 * kChunk);
+    const uint16_t* b_st = a_st + kChunk;
+    const int64_t left = V - k * kChunk;
+    uint4 va[kU], vb[kU];
+    uint32_t dep = 0;
+    if (left >= kChunk) {
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        va[u] = *reinterpret_cast<const uint4*>(a_st + 8 * (ct + u * Cfg::kConsumers));
+        vb[u] = *reinterpret_cast<const uint4*>(b_st + 8 * (ct + u * Cfg::kConsumers));
+        dep ^= va[u].x ^ va[u].y ^ va[u].z ^ va[u].w ^ vb[u].x ^ vb[u].y ^ vb[u].z ^ vb[u].w;
+      }
+    } else {
+      const int units = static_cast<int>(left / 8);
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int unit = ct + u * Cfg::kConsumers;
+        if (unit < units) {
+          va[u] = *reinterpret_cast<const uint4*>(a_st + 8 * unit);
+          vb[u] = *reinterpret_cast<const uint4*>(b_st + 8 * unit);
+          dep ^= va[u].x ^ va[u].y ^ va[u].z ^ va[u].w ^ vb[u].x ^ vb[u].y ^ vb[u].z ^ vb[u].w;
+        }
+      }
+    }
+    dep = __reduce_or_sync(kFull, dep);
+    if (lane == 0) {
+      fence_proxy_async_smem();
+      mbar_arrive_after(&empty[s], dep);
+    }
+    ++seq;
+    if (left >= kChunk) {
+      f_full(va, vb);
+    } else {
+      const int units = static_cast<int>(left / 8);
+#pragma unroll
+      for (int u = 0; u < kU; ++u)
+        if (ct + u * Cfg::kConsumers < units) f_one(va[u], vb[u]);
+    }
+    return true;
+  };
+  // Reduce (statistics, EAR part) over the consumer warps; every warp ends
+  // with the same total.
+  auto reduce = [&](Part mine, Part& tot) -> bool {
+    mine = warp_reduce(mine, c);
+    Part* slot = parts + (nred & 1u) * kCW;
+    uint64_t* bar = &red[nred & 1u];
+    if (lane == 0) {
+      slot[warp] = mine;
+      mbar_arrive(bar);
+    }
+    if (!ring_wait(bar, (nred >> 1) & 1u, abort)) return false;
+    ++nred;
+    tot = (lane < kCW) ? slot[lane] : none;
+    tot = warp_reduce(tot, c);
+    return true;
+  };
+
+  bool ok = true;
+  for (int64_t t = blockIdx.x; t < T && ok; t += G) {
+    VecStat vs = vec_stat_init(c);
+    for (int64_t k = 0; k < nch && ok; ++k)
+      ok = consume(
+          k, [&](const uint4(&va)[kU], const uint4(&vb)[kU]) { push_units<kU>(vs, va, vb, c); },
+          [&](const uint4& a1, const uint4& b1) {
+            const uint4 va[1] = {a1}, vb[1] = {b1};
+            push_units<1>(vs, va, vb, c);
+          });
+    Part tot;
+    if (!ok || !reduce(Part{vec_stat_final(vs, c), ear_part}, tot)) {
+      ok = false;
+      break;
+    }
+    if (ct == 0) {
+      if (t_prev >= 0) ear_tok[t_prev] = tot.ear;
+      kl_tok[t] = kl_of(tot.st, inv_temp);
+    }
+    const uint64_t c2 = pk(c, c);
+    const float nla = -lg2(tot.st.a.s), nlb = -lg2(tot.st.b.s);
+    const uint64_t ma2 = pk(tot.st.a.m, tot.st.a.m), mb2 = pk(tot.st.b.m, tot.st.b.m);
+    const uint64_t nla2 = pk(nla, nla), nlb2 = pk(nlb, nlb);
+    uint64_t acc[2] = {0ull, 0ull};
+    for (int64_t k = 0; k < nch && ok; ++k)
+      ok = consume(
+          k,
+          [&](const uint4(&va)[kU], const uint4(&vb)[kU]) {
+            ear_units<kU>(acc, va, vb, c2, ma2, nla2, mb2, nlb2);
+          },
+          [&](const uint4& a1, const uint4& b1) {
+            const uint4 va[1] = {a1}, vb[1] = {b1};
+            ear_units<1>(acc, va, vb, c2, ma2, nla2, mb2, nlb2);
+          });
+    ear_part = (pk_lo(acc[0]) + pk_hi(acc[0])) + (pk_lo(acc[1]) + pk_hi(acc[1]));
+    t_prev = t;
+  }
+  if (ok && t_prev >= 0) {
+    Part tot;
+    if (reduce(Part{none.st, ear_part}, tot)) {
+      if (ct == 0) ear_tok[t_prev] = tot.ear;
+    } else {
+      ok = false;
+    }
+  }
+  if (!ok && ct == 0 && flags) atomicOr(flags, kFlagTimeout);
+}
+
+template <int kCW, int kU, int kStages>
+constexpr size_t ring_smem_bytes() {
+  return static_cast<size_t>(kStages) * RingCfg<kCW, kU>::kStageBytes +
+         (2 * kStages + 2) * sizeof(uint64_t) + 2 * kCW * sizeof(Part) + 16;
+}
+
+// ---------------------------------------------------------------------------
+// Any V (the V % 8 != 0 case): one row per CTA, scalar loads; pass 1 the
+// online statistics, pass 2 the EAR terms (the row is back from L2).
+// ---------------------------------------------------------------------------
+template <int kThreads>
 __global__ void __launch_bounds__(kThreads)
     ear_kl_rows_kernel(const uint16_t* __restrict__ A, const uint16_t* __restrict__ Bq, int64_t T,
                        int64_t V, float c, float inv_temp, float* __restrict__ ear_tok,
@@ -159,240 +546,26 @@ __global__ void __launch_bounds__(kThreads)
     const uint16_t* a_row = A + t * V;
     const uint16_t* b_row = Bq + t * V;
     RowStat st{{-INFINITY, 0.0f}, {-INFINITY, 0.0f}, 0.0f};
-    if constexpr (kVec) {
-      const int64_t nv = V / 8;
-      for (int64_t i = threadIdx.x; i < nv; i += kThreads) {
-        const uint4 va = ld_stream_v4(a_row + 8 * i);
-        const uint4 vb = ld_stream_v4(b_row + 8 * i);
-        const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
-        const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          push(st, bf16_lo(wa[q]), bf16_lo(wb[q]), c);
-          push(st, bf16_hi(wa[q]), bf16_hi(wb[q]), c);
-        }
-      }
-    } else {
-      for (int64_t v = threadIdx.x; v < V; v += kThreads)
-        push(st, __uint_as_float(static_cast<uint32_t>(a_row[v]) << 16),
-             __uint_as_float(static_cast<uint32_t>(b_row[v]) << 16), c);
-    }
+    for (int64_t v = threadIdx.x; v < V; v += kThreads)
+      push(st, __uint_as_float(static_cast<uint32_t>(a_row[v]) << 16),
+           __uint_as_float(static_cast<uint32_t>(b_row[v]) << 16), c);
     const RowStat tot = block_reduce<kThreads>(st, c);
     const float la = lg2(tot.a.s), lb = lg2(tot.b.s);
     const float ma = tot.a.m, mb = tot.b.m;
-
-    // Pass 2: sum_v 2^min(u_v, w_v), four accumulators per thread.
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    if constexpr (kVec) {
-      const int64_t nv = V / 8;
-      for (int64_t i = threadIdx.x; i < nv; i += kThreads) {
-        const uint4 va = ld_ro_v4(a_row + 8 * i);
-        const uint4 vb = ld_ro_v4(b_row + 8 * i);
-        const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
-        const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          acc[q] += ex2(fminf((bf16_lo(wa[q]) - ma) * c - la, (bf16_lo(wb[q]) - mb) * c - lb));
-          acc[q] += ex2(fminf((bf16_hi(wa[q]) - ma) * c - la, (bf16_hi(wb[q]) - mb) * c - lb));
-        }
-      }
-    } else {
-      int q = 0;
-      for (int64_t v = threadIdx.x; v < V; v += kThreads) {
-        const float a = __uint_as_float(static_cast<uint32_t>(a_row[v]) << 16);
-        const float b = __uint_as_float(static_cast<uint32_t>(b_row[v]) << 16);
-        acc[q] += ex2(fminf((a - ma) * c - la, (b - mb) * c - lb));
-        q = (q + 1) & 3;
-      }
+    int q = 0;
+    for (int64_t v = threadIdx.x; v < V; v += kThreads) {
+      const float a = __uint_as_float(static_cast<uint32_t>(a_row[v]) << 16);
+      const float b = __uint_as_float(static_cast<uint32_t>(b_row[v]) << 16);
+      acc[q] += ex2(fminf((a - ma) * c - la, (b - mb) * c - lb));
+      q = (q + 1) & 3;
     }
     const float ear = block_sum<kThreads>((acc[0] + acc[1]) + (acc[2] + acc[3]));
     if (threadIdx.x == 0) {
-      constexpr float kLn2 = 0.693147180559945309f;
       ear_tok[t] = ear;
-      kl_tok[t] = (tot.w / tot.a.s) * inv_temp - ((ma - mb) * inv_temp + (la - lb) * kLn2);
+      kl_tok[t] = kl_of(tot, inv_temp);
     }
   }
-}
-
-// ---------------------------------------------------------------------------
-// Cluster kernel (V % 8 == 0): one HBM pass.  A cluster of CS CTAs (8, or 16
-// where the GPU allows it) owns one token row at a time; CTA r keeps slice r
-// of both logit rows in shared memory (double-buffered 1-D bulk copies: the
-// next row lands while this one is processed).  Per row: one pass of online
-// softmax statistics (running max with rescaling) -> one block reduction ->
-// the statistics are exchanged through distributed shared memory and merged
-// in rank order -> the EAR sum over the resident slice.  Rank 0 adds the EAR
-// partials of row i after the exchange of row i+1, so each row costs a single
-// cluster barrier.
-// ---------------------------------------------------------------------------
-constexpr int kClusterThreads = 512;
-
-struct SliceStat {
-  float ma, sa, w, mb, sb;
-};
-
-template <int CS>
-__global__ void __launch_bounds__(kClusterThreads)
-    ear_kl_cluster_kernel(const uint16_t* __restrict__ A, const uint16_t* __restrict__ Bq,
-                          int64_t T, int64_t V, int units_per_cta, float c, float inv_temp,
-                          float* __restrict__ ear_tok, float* __restrict__ kl_tok,
-                          uint32_t* __restrict__ flags) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  cg::cluster_group cluster = cg::this_cluster();
-  const int rank = static_cast<int>(cluster.block_rank());
-  const int64_t cluster_id = blockIdx.x / CS;
-  const int64_t nclusters = gridDim.x / CS;
-
-  const int64_t v8 = V / 8;
-  const int64_t r0 = static_cast<int64_t>(rank) * units_per_cta;
-  const int64_t u0 = r0 < v8 ? r0 : v8;
-  const int64_t u1 = (u0 + units_per_cta) < v8 ? (u0 + units_per_cta) : v8;
-  const int nu = static_cast<int>(u1 - u0);  // 16-byte units of this CTA's slice
-  const size_t slice_bytes = static_cast<size_t>(units_per_cta) * 16;
-
-  // [buf][tensor][slice] | barriers | stats[2] | ear[2] | merged
-  uint8_t* data = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(data + 4 * slice_bytes);
-  SliceStat* stats = reinterpret_cast<SliceStat*>(full + 2);
-  float* ear_part = reinterpret_cast<float*>(stats + 2);
-  SliceStat* merged = reinterpret_cast<SliceStat*>(ear_part + 2);
-  __shared__ int aborted;
-
-  const int64_t nrows = (T > cluster_id) ? (T - cluster_id + nclusters - 1) / nclusters : 0;
-
-  if (threadIdx.x == 0) {
-    mbar_init(&full[0], 1);
-    mbar_init(&full[1], 1);
-    aborted = 0;
-    fence_mbarrier_init();
-  }
-  __syncthreads();
-  cluster.sync();  // every CTA of the cluster is running before any remote access
-
-  auto issue = [&](int64_t i) {
-    const int buf = static_cast<int>(i & 1);
-    const int64_t t = cluster_id + i * nclusters;
-    const uint32_t bytes = static_cast<uint32_t>(nu) * 16;
-    mbar_arrive_expect_tx(&full[buf], 2 * bytes);
-    if (bytes) {
-      bulk_load(data + (2 * buf) * slice_bytes, A + t * V + u0 * 8, bytes, &full[buf]);
-      bulk_load(data + (2 * buf + 1) * slice_bytes, Bq + t * V + u0 * 8, bytes, &full[buf]);
-    }
-  };
-  int64_t issued = 0;
-  if (threadIdx.x == 0)
-    for (; issued < 2 && issued < nrows; ++issued) issue(issued);
-
-  for (int64_t i = 0; i < nrows; ++i) {
-    const int buf = static_cast<int>(i & 1);
-    const int64_t t = cluster_id + i * nclusters;
-    if (!aborted) {
-      if (!mbar_wait_bounded(&full[buf], static_cast<uint32_t>((i >> 1) & 1))) {
-        aborted = 1;
-        if (flags) atomicOr(flags, kFlagTimeout);
-      }
-    }
-    __syncthreads();
-    const bool live = !aborted;
-    const uint4* sa4 = reinterpret_cast<const uint4*>(data + (2 * buf) * slice_bytes);
-    const uint4* sb4 = reinterpret_cast<const uint4*>(data + (2 * buf + 1) * slice_bytes);
-
-    // One pass of online softmax statistics over the resident slice.
-    RowStat st{{-INFINITY, 0.0f}, {-INFINITY, 0.0f}, 0.0f};
-    if (live) {
-      for (int k = threadIdx.x; k < nu; k += kClusterThreads) {
-        const uint4 va = sa4[k], vb = sb4[k];
-        const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
-        const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          push(st, bf16_lo(wa[q]), bf16_lo(wb[q]), c);
-          push(st, bf16_hi(wa[q]), bf16_hi(wb[q]), c);
-        }
-      }
-    }
-    const RowStat tot = block_reduce<kClusterThreads>(st, c);
-    if (threadIdx.x == 0) stats[buf] = SliceStat{tot.a.m, tot.a.s, tot.w, tot.b.m, tot.b.s};
-
-    cluster.sync();  // statistics of row i (and EAR partials of row i-1) are visible
-
-    if (threadIdx.x < 32) {
-      // Merge the CS slices in rank order (lane 0 does the fixed-order sums).
-      SliceStat r = {-INFINITY, 0.0f, 0.0f, -INFINITY, 0.0f};
-      if (threadIdx.x < CS) r = cluster.map_shared_rank(stats, static_cast<int>(threadIdx.x))[buf];
-      float prev_ear = 0.0f;
-      if (rank == 0 && i > 0 && threadIdx.x < CS)
-        prev_ear = cluster.map_shared_rank(ear_part, static_cast<int>(threadIdx.x))[buf ^ 1];
-      float Ma = -INFINITY, Mb = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < CS; ++j) {
-        Ma = fmaxf(Ma, __shfl_sync(kFull, r.ma, j));
-        Mb = fmaxf(Mb, __shfl_sync(kFull, r.mb, j));
-      }
-      float Sa = 0.0f, Sb = 0.0f, W = 0.0f, E = 0.0f;
-#pragma unroll
-      for (int j = 0; j < CS; ++j) {
-        const float ma = __shfl_sync(kFull, r.ma, j), mb = __shfl_sync(kFull, r.mb, j);
-        const float sa = __shfl_sync(kFull, r.sa, j), sb = __shfl_sync(kFull, r.sb, j);
-        const float w = __shfl_sync(kFull, r.w, j);
-        E += __shfl_sync(kFull, prev_ear, j);
-        if (ma != -INFINITY) {
-          const float f = ex2((ma - Ma) * c);
-          Sa = fmaf(sa, f, Sa);
-          W = fmaf(w, f, W);
-        }
-        if (mb != -INFINITY) Sb = fmaf(sb, ex2((mb - Mb) * c), Sb);
-      }
-      if (threadIdx.x == 0) {
-        *merged = SliceStat{Ma, Sa, W, Mb, Sb};
-        if (rank == 0) {
-          constexpr float kLn2 = 0.693147180559945309f;
-          if (live)
-            kl_tok[t] = (W / Sa) * inv_temp - ((Ma - Mb) * inv_temp + (lg2(Sa) - lg2(Sb)) * kLn2);
-          if (i > 0) ear_tok[t - nclusters] = E;
-        }
-      }
-    }
-    __syncthreads();
-    const SliceStat g = *merged;
-    const float la = lg2(g.sa), lb = lg2(g.sb);
-
-    // EAR terms of the resident slice: sum 2^min(log2 p, log2 q).
-    float e_acc[2] = {0.0f, 0.0f};
-    if (live) {
-      for (int k = threadIdx.x; k < nu; k += kClusterThreads) {
-        const uint4 va = sa4[k], vb = sb4[k];
-        const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
-        const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          e_acc[q & 1] += ex2(fminf((bf16_lo(wa[q]) - g.ma) * c - la, (bf16_lo(wb[q]) - g.mb) * c - lb));
-          e_acc[q & 1] += ex2(fminf((bf16_hi(wa[q]) - g.ma) * c - la, (bf16_hi(wb[q]) - g.mb) * c - lb));
-        }
-      }
-    }
-    const float es = block_sum<kClusterThreads>(e_acc[0] + e_acc[1]);
-    if (threadIdx.x == 0) ear_part[buf] = es;
-    // block_sum ended with __syncthreads: every read of this buffer is done.
-    if (threadIdx.x == 0 && !aborted && issued < nrows && issued == i + 2) {
-      fence_proxy_async_smem();
-      issue(issued);
-      ++issued;
-    }
-  }
-  cluster.sync();  // EAR partials of the last row are visible
-  if (rank == 0 && threadIdx.x == 0 && nrows > 0) {
-    const int buf = static_cast<int>((nrows - 1) & 1);
-    float e = 0.0f;
-    for (int j = 0; j < CS; ++j) e += cluster.map_shared_rank(ear_part, j)[buf];
-    ear_tok[cluster_id + (nrows - 1) * nclusters] = e;
-  }
-  // Copies issued but never consumed (only after a timeout) must land first.
-  if (threadIdx.x == 0 && aborted) {
-    for (int64_t i = (issued > 2 ? issued - 2 : 0); i < issued; ++i)
-      mbar_wait_bounded(&full[i & 1], static_cast<uint32_t>((i >> 1) & 1));
-  }
-  cluster.sync();  // keep shared memory alive until rank 0 has read it
 }
 
 // Means over tokens in binary64, one block, fixed summation order.
@@ -421,55 +594,6 @@ __global__ void __launch_bounds__(1024)
   }
 }
 
-constexpr size_t kClusterSmemExtra = 16 + 2 * sizeof(SliceStat) + 8 + sizeof(SliceStat) + 64;
-
-// Launch the cluster kernel with CS CTAs per cluster if the GPU can keep such
-// clusters resident; returns the number of resident CTAs it would use (0 if
-// the configuration is impossible) and launches only when `launch` is set.
-template <int CS>
-int64_t cluster_launch(bool launch, const uint16_t* a, const uint16_t* b, int64_t T, int64_t V,
-                       float c, float inv_temp, float* ear_tok, float* kl_tok, uint32_t* flags,
-                       cudaStream_t stream, cudaError_t* err) {
-  const int64_t v8 = V / 8;
-  const int64_t upc = (v8 + CS - 1) / CS;
-  const size_t smem = static_cast<size_t>(4 * upc * 16) + kClusterSmemExtra;
-  if (smem > 220 * 1024) return 0;
-  if (cudaFuncSetAttribute(ear_kl_cluster_kernel<CS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess) {
-    cudaGetLastError();
-    return 0;
-  }
-  if (CS > 8 && cudaFuncSetAttribute(ear_kl_cluster_kernel<CS>,
-                                     cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
-    cudaGetLastError();
-    return 0;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(kClusterThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CS;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cfg.gridDim = dim3(CS * 32, 1, 1);
-  int max_clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&max_clusters, ear_kl_cluster_kernel<CS>, &cfg) != cudaSuccess)
-    max_clusters = 0;
-  cudaGetLastError();
-  if (max_clusters <= 0) return 0;
-  const int64_t nc = T < max_clusters ? T : max_clusters;
-  if (launch) {
-    cfg.gridDim = dim3(static_cast<unsigned>(CS * nc), 1, 1);
-    *err = cudaLaunchKernelEx(&cfg, ear_kl_cluster_kernel<CS>, a, b, T, V, static_cast<int>(upc),
-                              c, inv_temp, ear_tok, kl_tok, flags);
-  }
-  return static_cast<int64_t>(max_clusters) * CS;
-}
-
 }  // namespace
 
 cudaError_t launch_ear_kl(const uint16_t* a, const uint16_t* b, int64_t T, int64_t V,
@@ -482,35 +606,27 @@ cudaError_t launch_ear_kl(const uint16_t* a, const uint16_t* b, int64_t T, int64
   const float c = 1.4426950408889634f * inv_temp;
   cudaError_t err = cudaSuccess;
 
-  // Single-pass cluster kernel when rows are 16-byte aligned and the slices
-  // fit in shared memory; the configuration with more resident CTAs wins
-  // (16-CTA clusters halve the slice, so two CTAs can share an SM).  The row
-  // kernel covers every other case.
-  bool done = false;
-  if (V % 8 == 0) {
-    const int64_t r16 = cluster_launch<16>(false, a, b, T, V, c, inv_temp, ear_tok, kl_tok, flags, stream, &err);
-    const int64_t r8 = cluster_launch<8>(false, a, b, T, V, c, inv_temp, ear_tok, kl_tok, flags, stream, &err);
-    if (r16 > 0 && r16 >= r8) {
-      cluster_launch<16>(true, a, b, T, V, c, inv_temp, ear_tok, kl_tok, flags, stream, &err);
-      done = true;
-    } else if (r8 > 0) {
-      cluster_launch<8>(true, a, b, T, V, c, inv_temp, ear_tok, kl_tok, flags, stream, &err);
-      done = true;
-    }
+  const bool aligned = ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b)) & 15u) == 0;
+  if (V % 8 == 0 && aligned) {
+    constexpr int kCW = kEarConsumerWarps, kU = kEarUnits, kS = kEarStages;
+    constexpr size_t smem = ring_smem_bytes<kCW, kU, kS>();
+    static_assert(smem <= 227 * 1024, "ring exceeds shared memory");
+    auto kern = ear_kl_ring_kernel<kCW, kU, kS>;
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
     if (err != cudaSuccess) return err;
+    const int64_t cap = static_cast<int64_t>(sms);
+    const int64_t blocks = T < cap ? T : cap;
+    kern<<<static_cast<unsigned>(blocks), RingCfg<kCW, kU>::kThreads, smem, stream>>>(
+        a, b, T, V, c, inv_temp, ear_tok, kl_tok, flags);
+  } else {
+    const int64_t cap = static_cast<int64_t>(sms);
+    const int64_t blocks = T < cap ? T : cap;
+    ear_kl_rows_kernel<1024><<<static_cast<unsigned>(blocks), 1024, 0, stream>>>(
+        a, b, T, V, c, inv_temp, ear_tok, kl_tok);
   }
-  if (!done) {
-    constexpr int kThreads = 1024;
-    const int64_t blocks = T < static_cast<int64_t>(sms) * 2 ? T : static_cast<int64_t>(sms) * 2;
-    if (V % 8 == 0)
-      ear_kl_rows_kernel<kThreads, true><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
-          a, b, T, V, c, inv_temp, ear_tok, kl_tok);
-    else
-      ear_kl_rows_kernel<kThreads, false><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
-          a, b, T, V, c, inv_temp, ear_tok, kl_tok);
-    err = cudaGetLastError();
-    if (err != cudaSuccess) return err;
-  }
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
   if (ear_mean || kl_mean) {
     token_mean_kernel<<<1, 1024, 0, stream>>>(ear_tok, kl_tok, T, ear_mean, kl_mean);
     err = cudaGetLastError();
