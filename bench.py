@@ -16,6 +16,16 @@ sweep N=K=8192 at every b, the tiled GEMM at prefill sizes, and EAR/KL over
 pages' models (no checkpoints or datasets here).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl slq|reference]
+  python bench.py --case SPEC [--steps K] [--warmup W]
+
+--case runs one kernel of the path on its own (W untimed launches, then K
+timed ones) and prints {"case", "avg_us", ...}: the command the profiles'
+ncu captures use.  SPEC is one of
+  block                     the 21 decode launches of the Qwen3-8B block
+  decode:N:K:b:M            one decode-path dequant-GEMM
+  tiled:N:K:b:M             one tiled-path dequant-GEMM
+  ear:T:V:tau               one EAR/KL reduction
+  quantize:N:K:b            one quantize+pack
 
 --impl reference times the CPU oracle (the plain reference implementation
 of the same arithmetic) on a bounded sample of the same workload, on the
@@ -352,7 +362,7 @@ def run_slq(args, rank, world, local_rank):
             },
             "roofline": {
                 "bound": "hbm",
-                "kernel": "gemm_decode_kernel<b> (TMA-staged packed W dequantized into TMEM, tcgen05.mma with the TMEM A operand, persistent stream-K over one CTA per SM; M<=16)",
+                "kernel": "gemm_decode_kernel<b> (TMA-streamed packed W dequantized in registers into mma.sync A fragments, fp32 group-scaled accumulate, persistent stream-K over two CTAs per SM with a deterministic split-K fixup; M<=16)",
                 "achieved": round(achieved, 1),
                 "peak": hbm_peak,
                 "unit": "GB/s",
@@ -360,7 +370,7 @@ def run_slq(args, rank, world, local_rank):
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6650 GB/s",
                 "algorithmic_bytes": "N*K*(b/8 + 3/128) per launch (codes + fp16 scale + u8 zero)",
                 "avg_launch_us": round(kernel_ms * 1e3, 3) if kernel_ms else None,
-                "traffic": None,
+                "traffic": decode_traffic(),
                 "per_M": breakdown,
             },
             "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
@@ -553,6 +563,90 @@ def run_reference(args, rank, world):
     }
 
 
+def decode_traffic():
+    """DRAM bytes per decode launch of this workload from the committed ncu
+    capture (profiles/decode_block_traffic.json), or None when the kernel
+    source has changed since it was taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "decode_block_traffic.json")
+    src = os.path.join(ROOT, "weight_only_mixed_b200", "csrc", "gemm_decode.cu")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except (OSError, ValueError):
+        return None
+    if rec.get("gemm_decode_cu_sha256") != sha:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def run_case(args):
+    """One kernel of the path, launched on its own (for ncu captures)."""
+    import torch
+    import synth
+    import weight_only_mixed_b200 as slq
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+    kind, *parts = args.case.split(":")
+    vals = [float(p) if "." in p else int(p) for p in parts]
+    if kind == "block":
+        items = []
+        for M in DECODE_MS:
+            for i, (_, N, K, b) in enumerate(QWEN3_8B_BLOCK):
+                qw = slq.quantize(synth.weights_torch(N, K, seed=synth.SEED_WEIGHTS + 10 * i, device=dev), b)
+                x = synth.activations_torch(M, K, seed=synth.SEED_X + 10 * i + M, device=dev)
+                y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+                items.append((x, qw, y))
+
+        def fn():
+            for x, qw, y in items:
+                slq.gemm(x, qw, out=y, stream=stream)
+        per_call = len(items)
+    elif kind in ("decode", "tiled"):
+        N, K, b, M = vals
+        qw = slq.quantize(synth.weights_torch(N, K, device=dev), b)
+        x = synth.activations_torch(M, K, device=dev)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+
+        def fn():
+            slq.gemm(x, qw, out=y, path=kind, stream=stream)
+        per_call = 1
+    elif kind == "ear":
+        T, V, tau = vals
+        a, bq = synth.logits_torch(T, V, device=dev)
+
+        def fn():
+            slq.ear_kl(a, bq, float(tau), stream=stream)
+        per_call = 2  # the reduction and the token means
+    elif kind == "quantize":
+        N, K, b = vals
+        W = synth.weights_torch(N, K, device=dev)
+        q = slq.empty_quantized(N, K, b, dev)
+
+        def fn():
+            slq.quantize(W, b, out=q, stream=stream)
+        per_call = 1
+    else:
+        raise SystemExit(f"unknown --case {args.case}")
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        fn()
+    e1.record(stream)
+    e1.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / max(1, args.steps)
+    print(json.dumps({"case": args.case, "avg_us_per_call": round(us, 3), "launches_per_call": per_call,
+                      "calls": args.steps, "warmup": args.warmup}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -563,7 +657,11 @@ def main():
     ap.add_argument("--headline-only", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=512)
+    ap.add_argument("--case", default=None, help="run one kernel on its own (see the module docstring)")
     args = ap.parse_args()
+    if args.case:
+        run_case(args)
+        return
     assert args.warmup >= 3 or args.impl == "reference", "at least 3 warm-up steps"
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -54,16 +54,22 @@ enum {
   SLQ_FLAG_TIMEOUT = 4u         /* a bounded on-chip wait gave up; outputs are unspecified */
 };
 
-/* GEMM kernel choice for slq_gemm_ex.  Both kernels dequantize the weights
- * to exact bf16 (q - z), multiply on the tcgen05 tensor cores with fp32
- * accumulation in TMEM, one product per 128-wide group, and apply the fp16
- * group scale to that fp32 product. */
+/* GEMM kernel choice for slq_gemm_ex.  Every kernel forms exact bf16 values
+ * from the codes, multiplies on the tensor cores with fp32 accumulation, one
+ * product per 128-wide group, and applies the fp16 group scale to that fp32
+ * product; they differ in how the work is split. */
 typedef enum {
-  SLQ_GEMM_AUTO = 0,   /* DECODE for M <= 16, TILED above */
-  SLQ_GEMM_DECODE = 1, /* M <= 16: weights dequantized into TMEM, one persistent CTA per SM,
-                          the row tiles x groups split evenly over the CTAs (needs a workspace) */
-  SLQ_GEMM_TILED = 2   /* any M >= 1: 128 x {64, 128, 256} output tiles, weights dequantized
-                          into shared memory, K split over a thread-block cluster for M <= 64 */
+  SLQ_GEMM_AUTO = 0,   /* GEMV for M <= 16, TILED above */
+  SLQ_GEMM_DECODE = 1, /* M <= 16: packed weights streamed by TMA, dequantized in registers
+                          into mma.sync fragments, the row tiles x groups split evenly over
+                          two CTAs per SM (stream-K; needs a workspace) */
+  SLQ_GEMM_TILED = 2,  /* any M >= 1: 128 x {64, 128, 256} output tiles, weights dequantized
+                          into shared memory, tcgen05.mma into TMEM, K split over a
+                          thread-block cluster for M <= 64 */
+  SLQ_GEMM_GEMV = 3    /* M <= 16: one CTA per 16- or 32-row tile whose warps split K, packed
+                          weights streamed with cp.async into per-warp shared-memory rings,
+                          dequantized in registers into mma.sync fragments; partial tiles
+                          added in shared memory (no workspace) */
 } slq_gemm_path;
 
 /* Group size along K, fixed by the format ("asymmetric INT, group size 128",
@@ -84,14 +90,16 @@ const char *slq_status_string(slq_status status);
  * Returns 0 for invalid arguments. */
 size_t slq_packed_words(int64_t N, int64_t K, int bits);
 
-/* Which kernel slq_gemm would run for these sizes (SLQ_GEMM_DECODE or
+/* Which kernel slq_gemm would run for these sizes (SLQ_GEMM_GEMV or
  * SLQ_GEMM_TILED).  Host-only; launches nothing. */
 slq_gemm_path slq_gemm_select(int64_t M, int64_t N, int64_t K, int bits);
 
-/* Bytes of device workspace slq_gemm needs for Y[M, N] = X[M, K] W[N, K]^T
- * on the CURRENT device (the decode kernel splits the layer over that
- * device's SMs); 0 when the call needs none (M > 16, or every row tile falls
- * in one CTA).  Returns 0 for invalid arguments.
+/* Bytes of device workspace the SLQ_GEMM_DECODE kernel needs for
+ * Y[M, N] = X[M, K] W[N, K]^T on the CURRENT device (it splits the layer over
+ * that device's SMs); 0 when it needs none (every row tile falls in one CTA)
+ * and for M > 16.  The kernels slq_gemm selects (GEMV, TILED) need no
+ * workspace, so a buffer of this size serves every path.  Returns 0 for
+ * invalid arguments.
  *
  * Workspace rules: device memory owned by the caller, 256-byte aligned, not
  * overlapping any other argument.  Its first 64 KiB hold per-row-tile
@@ -163,9 +171,10 @@ slq_status slq_gemm(const void *X_bf16, int64_t M, int64_t N, int64_t K,
                     void *workspace, size_t workspace_bytes, uint32_t *flags,
                     void *stream);
 
-/* slq_gemm with an explicit kernel choice (SLQ_GEMM_DECODE needs M <= 16;
- * the workspace requirement is that of the chosen kernel: none for
- * SLQ_GEMM_TILED).  Same arguments and results otherwise. */
+/* slq_gemm with an explicit kernel choice (SLQ_GEMM_DECODE and SLQ_GEMM_GEMV
+ * need M <= 16; only SLQ_GEMM_DECODE needs a workspace, of
+ * slq_gemm_workspace_bytes bytes, and takes N <= 2097152).  Same arguments
+ * and results otherwise. */
 slq_status slq_gemm_ex(const void *X_bf16, int64_t M, int64_t N, int64_t K,
                        int bits, const uint32_t *packed,
                        const void *scales_f16, const uint8_t *zeros, void *Y,
@@ -190,8 +199,9 @@ slq_status slq_gemm_ex(const void *X_bf16, int64_t M, int64_t N, int64_t K,
  *
  * Arguments, layouts and results are those of slq_gemm, without workspace.
  *   M            0..16; larger M gives SLQ_ERR_INVALID_ARGUMENT.
- *   Layers whose decode workspace (slq_gemm_workspace_bytes) exceeds
- *   SLQ_DECODE_STATIC_SCRATCH_BYTES give SLQ_ERR_INVALID_ARGUMENT.
+ *   It runs the SLQ_GEMM_DECODE kernel; layers whose workspace for it
+ *   (slq_gemm_workspace_bytes) exceeds SLQ_DECODE_STATIC_SCRATCH_BYTES give
+ *   SLQ_ERR_INVALID_ARGUMENT.
  *
  * Every call shares the one array of its device: calls that may run at the
  * same time on the GPU (different streams, or several host threads) race on

@@ -56,8 +56,8 @@ def test_packed_words():
 
 
 def test_gemm_select():
-    assert slq.gemm_select(1, 4096, 4096, 4) == "decode"
-    assert slq.gemm_select(16, 4096, 4096, 4) == "decode"
+    assert slq.gemm_select(1, 4096, 4096, 4) == "gemv"
+    assert slq.gemm_select(16, 4096, 4096, 4) == "gemv"
     assert slq.gemm_select(17, 4096, 4096, 4) == "tiled"
     assert slq.gemm_select(4096, 8192, 8192, 2) == "tiled"
 
@@ -93,7 +93,7 @@ def test_gemm_validation():
     bad = [dict(bits=1), dict(bits=9), dict(K=64), dict(K=129), dict(M=-1), dict(N=-1),
            dict(X=None), dict(Y=None), dict(packed=None), dict(scales=None), dict(zeros=None),
            dict(X=FAKE + 2), dict(Y=FAKE + (4 << 24) + 8), dict(packed=FAKE + (1 << 24) + 4),
-           dict(dtype=2), dict(path=3), dict(path=1, M=17), dict(Y=FAKE + 16),  # Y overlaps X
+           dict(dtype=2), dict(path=4), dict(path=1, M=17), dict(path=3, M=17), dict(Y=FAKE + 16),  # Y overlaps X
            dict(M=1 << 31)]
     for kw in bad:
         assert _g(**kw) == slq.SLQ_ERR_INVALID_ARGUMENT, kw
@@ -107,15 +107,16 @@ def test_gemm_workspace_rules():
     assert need > 0
     assert slq.gemm_workspace_bytes(17, N, K, b) == 0  # tiled kernel: none
     assert slq.gemm_workspace_bytes(4, N, 100, b) == 0  # invalid K
-    kw = dict(M=M, N=N, K=K, bits=b)
+    kw = dict(M=M, N=N, K=K, bits=b, path=1)  # the stream-K decode kernel
     big = dict(packed=FAKE + (1 << 28), scales=FAKE + (2 << 28), zeros=FAKE + (3 << 28),
                Y=FAKE + (4 << 28), ws=FAKE + (5 << 28))
     for bad in [dict(ws=None), dict(ws_bytes=need - 1), dict(ws=FAKE + (5 << 28) + 16),
                 dict(ws=FAKE + 256)]:  # misaligned, overlapping X
         args = {**kw, **big, "ws_bytes": need, **bad}
         assert _g(**args) == slq.SLQ_ERR_INVALID_ARGUMENT, bad
-    # The tiled kernel ignores the workspace.
-    assert _g(**{**kw, **big, "ws": None, "ws_bytes": 0, "path": 2}) != slq.SLQ_ERR_INVALID_ARGUMENT
+    # The tiled and GEMV kernels (and AUTO, which picks them) take none.
+    for path in (0, 2, 3):
+        assert _g(**{**kw, **big, "ws": None, "ws_bytes": 0, "path": path}) != slq.SLQ_ERR_INVALID_ARGUMENT
 
 
 def _e(T=4, V=1000, tau=1.0, a=FAKE, b=FAKE + (1 << 24), ear=FAKE + (2 << 24),

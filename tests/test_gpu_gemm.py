@@ -59,16 +59,17 @@ DECODE_SHAPES = [(1, 1, 128), (2, 7, 256), (3, 33, 384), (5, 100, 1152), (8, 100
                  (9, 64, 2048), (15, 48, 128 * 9), (16, 256, 4096), (4, 300, 128 * 35)]
 
 
+@pytest.mark.parametrize("path", ["gemv", "decode"])
 @pytest.mark.parametrize("bits", BITS)
 @pytest.mark.parametrize("M,N,K", DECODE_SHAPES)
-def test_decode_matches_oracle(bits, M, N, K):
+def test_decode_matches_oracle(bits, M, N, K, path):
     host, qw = _layer(N, K, bits, seed=M * 7 + N + K + bits)
     x = synth.activations(M, K, seed=M + K)
-    _check(x, host, qw, "decode")
+    _check(x, host, qw, path)
 
 
 @pytest.mark.parametrize("bits", BITS)
-@pytest.mark.parametrize("path", ["decode", "tiled"])
+@pytest.mark.parametrize("path", ["gemv", "decode", "tiled"])
 def test_one_hot_rows_are_exact(bits, path):
     N, K = 40, 512
     host, qw = _layer(N, K, bits, seed=77 + bits)

@@ -41,8 +41,10 @@ SLQ_FLAG_TIMEOUT = 4
 SLQ_GEMM_AUTO = 0
 SLQ_GEMM_DECODE = 1
 SLQ_GEMM_TILED = 2
+SLQ_GEMM_GEMV = 3
 
-_PATHS = {"auto": SLQ_GEMM_AUTO, "decode": SLQ_GEMM_DECODE, "tiled": SLQ_GEMM_TILED}
+_PATHS = {"auto": SLQ_GEMM_AUTO, "decode": SLQ_GEMM_DECODE, "tiled": SLQ_GEMM_TILED,
+          "gemv": SLQ_GEMM_GEMV}
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -110,7 +112,8 @@ def packed_words(N: int, K: int, bits: int) -> int:
 
 
 def gemm_select(M: int, N: int, K: int, bits: int) -> str:
-    return {SLQ_GEMM_DECODE: "decode", SLQ_GEMM_TILED: "tiled"}[_lib.slq_gemm_select(M, N, K, bits)]
+    return {SLQ_GEMM_DECODE: "decode", SLQ_GEMM_TILED: "tiled",
+            SLQ_GEMM_GEMV: "gemv"}[_lib.slq_gemm_select(M, N, K, bits)]
 
 
 def gemm_workspace_bytes(M: int, N: int, K: int, bits: int) -> int:
@@ -203,9 +206,7 @@ def gemm(X, qw: QuantizedWeight, out_dtype=None, path: str = "auto", out=None, f
     assert K == qw.K
     y = out if out is not None else torch.empty((M, qw.N), dtype=out_dtype, device=X.device)
     dt = SLQ_DTYPE_F32 if y.dtype == torch.float32 else SLQ_DTYPE_BF16
-    need = 0
-    if path != "tiled":
-        need = gemm_workspace_bytes(M, qw.N, K, qw.bits) if path == "auto" or M <= 16 else 0
+    need = gemm_workspace_bytes(M, qw.N, K, qw.bits) if path == "decode" else 0
     ws = workspace if workspace is not None else workspace_for(need, stream)
     ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check(_lib.slq_gemm_ex(_ptr(X), M, qw.N, K, qw.bits, _ptr(qw.packed), _ptr(qw.scales),

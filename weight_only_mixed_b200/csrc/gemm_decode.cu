@@ -660,6 +660,284 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 }
 
 // ---------------------------------------------------------------------------
+// Split-K GEMV (M <= 16) without workspace.  A CTA owns 16 * RT consecutive
+// weight rows; its S warps split the rows' groups into S contiguous K ranges.
+// Each warp streams its rows' groups (16b bytes per row and group) through a
+// private D-stage shared-memory ring with 16-byte cp.async copies, GB groups
+// per stage, so D - 1 stages are in flight per warp without holding
+// registers.  A thread then reads its 4b-byte unit of each of its 2 * RT rows
+// and feeds the pairs to mma.sync as above; the activation fragments come
+// through L1; the S partial tiles are added in shared memory in warp order
+// (deterministic, no cross-CTA step).
+//
+// For b = 3, 5, 6, 7 (codes cut by word boundaries, the costliest to unpack)
+// the zero point leaves the inner loop: the A pairs are the exact bf16 values
+// 128 + q (q < 128), one more mma per k-step with an all-ones A gives
+// sum_k x over the group, and the group's product is
+// s * (sum (128 + q) x - (128 + z) sum x).  For b = 2, 4, 8 the pairs are
+// (q - z) as above.
+// ---------------------------------------------------------------------------
+template <int B>
+__device__ __forceinline__ void lds_unit(const uint8_t* p, uint32_t (&w)[B]) {
+  if constexpr (B == 4 || B == 8) {
+#pragma unroll
+    for (int i = 0; i < B / 4; ++i) {
+      const uint4 v = *reinterpret_cast<const uint4*>(p + 16 * i);
+      w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+    }
+  } else if constexpr (B == 2 || B == 6) {
+#pragma unroll
+    for (int i = 0; i < B / 2; ++i) {
+      const uint2 v = *reinterpret_cast<const uint2*>(p + 8 * i);
+      w[2 * i] = v.x; w[2 * i + 1] = v.y;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < B; ++i) w[i] = reinterpret_cast<const uint32_t*>(p)[i];
+  }
+}
+
+// Pair p of a unit as exact bf16 (128 + q_2p, 128 + q_2p+1), b <= 7.
+template <int B>
+__device__ __forceinline__ uint32_t pair_raw(const uint32_t (&w)[B], int p) {
+  if constexpr (B == 4) {
+    const uint32_t y = __byte_perm(w[p >> 2], 0u, 0x4440 | (p & 3)) * 0x1001u;
+    return (y & 0x000F000Fu) | 0x43004300u;
+  } else if constexpr (B == 2) {
+    const uint32_t y = __byte_perm(w[p >> 3], 0u, 0x4440 | ((p >> 1) & 3)) * 0x4001u;
+    return ((y >> (4 * (p & 1))) & 0x00030003u) | 0x43004300u;
+  } else {
+    return dq::code_at<B>(w, 2 * p) | (dq::code_at<B>(w, 2 * p + 1) << 16) | 0x43004300u;
+  }
+}
+
+__device__ __forceinline__ uint32_t ld_ro_u16(const void* p) {
+  unsigned short r;
+  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(r) : "l"(p));
+  return r;
+}
+__device__ __forceinline__ uint32_t ld_ro_u8(const void* p) {
+  unsigned short r;
+  asm volatile("ld.global.nc.u8 %0, [%1];" : "=h"(r) : "l"(p));
+  return r & 0xFFu;
+}
+
+template <int B, int RT, int GB>
+constexpr int gemv_stage_bytes() {  // one warp's stage
+  return GB * RT * 2 * 8 * 16 * B;
+}
+
+template <int B, int NT, int RT, int S, int GB, int D>
+__global__ void __launch_bounds__(32 * S)
+    gemm_gemv_kernel(const uint16_t* __restrict__ X, int M, int N, int K,
+                     const uint8_t* __restrict__ packed, const uint16_t* __restrict__ scales,
+                     const uint8_t* __restrict__ zeros, void* __restrict__ Y, int y_f32, int gmax) {
+  constexpr int kTile = 16 * RT;
+  constexpr int kRowG = 16 * B;  // bytes of one row's group
+  constexpr int kStage = gemv_stage_bytes<B, RT, GB>();
+  constexpr bool kFold = B == 3 || B == 5 || B == 6 || B == 7;
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = lane & 3, q = lane >> 2;
+  const int G = K / kGroup;
+  const int64_t row_bytes = static_cast<int64_t>(G) * kRowG;
+  const int tile0 = static_cast<int>(blockIdx.x) * kTile;
+  const int g0 = static_cast<int>(static_cast<int64_t>(G) * warp / S);
+  const int g1 = static_cast<int>(static_cast<int64_t>(G) * (warp + 1) / S);
+  const int ng = g1 - g0;
+  uint8_t* ring = smem + warp * (D * kStage);
+  uint32_t* szs = reinterpret_cast<uint32_t*>(smem + S * D * kStage) + warp * (kTile * gmax);
+
+  // Rows of this thread: 16 rt + q + 8 h of the tile (clamped for loads).
+  // Stage layout: [group i][rt][h][q][16b bytes]; the quad (same q) copies
+  // its row's group as b 16-byte chunks, chunk c by lane t = c % 4.
+  const uint8_t* wrow[RT][2];
+#pragma unroll
+  for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      wrow[rt][h] = packed + min(tile0 + 16 * rt + q + 8 * h, N - 1) * row_bytes;
+  auto issue = [&](int stage, int gb) {
+    uint8_t* st = ring + stage * kStage + q * kRowG;
+#pragma unroll
+    for (int i = 0; i < GB; ++i)
+      if (gb + i < g1) {
+#pragma unroll
+        for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int c = t; c < B; c += 4)
+              cp_async_16(st + ((i * RT + rt) * 2 + h) * 8 * kRowG + 16 * c,
+                          wrow[rt][h] + (gb + i) * kRowG + 16 * c, 16u);
+      }
+  };
+
+  // The first stage's weights go to L2 while the previous kernel finishes;
+  // nothing is read into the SM before it has completed.
+  if (ng > 0) {
+#pragma unroll
+    for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) asm volatile("prefetch.global.L2 [%0];" ::"l"(wrow[rt][h] + g0 * kRowG));
+  }
+  grid_dependency_wait();
+  const int nb = (ng + GB - 1) / GB;
+#pragma unroll
+  for (int d = 0; d < D - 1; ++d) {
+    if (d < nb) issue(d, g0 + d * GB);
+    cp_async_commit();
+  }
+  // This warp's scales and zeros, (scale | zero << 16) per (row, group).
+  for (int idx = lane; idx < kTile * ng; idx += 32) {
+    const int r = idx / ng, gg = idx - r * ng;
+    const int64_t o = static_cast<int64_t>(min(tile0 + r, N - 1)) * G + g0 + gg;
+    szs[r * gmax + gg] = ld_ro_u16(scales + o) | (ld_ro_u8(zeros + o) << 16);
+  }
+  __syncwarp();
+
+  float acc[RT][NT][4];
+#pragma unroll
+  for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[rt][nt][e] = 0.0f;
+
+  for (int bi = 0; bi < nb; ++bi) {
+    const int nx = bi + D - 1;
+    if (nx < nb) issue(nx % D, g0 + nx * GB);
+    cp_async_commit();
+    cp_async_wait<D - 1>();
+    __syncwarp();  // the quad's chunks of every row are in
+    const uint8_t* st = ring + (bi % D) * kStage + q * kRowG + 4 * B * t;
+#pragma unroll
+    for (int i = 0; i < GB; ++i) {
+      const int gl = bi * GB + i;  // group index within this warp's range
+      if (gl >= ng) break;
+      const int g = g0 + gl;
+      // Activation fragments: X[n][128 g + 32 t + 4 j .. + 3] for k-step j.
+      uint4 xv[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int n = q + 8 * nt;
+        const uint16_t* xp = X + static_cast<int64_t>(n) * K + g * kGroup + 32 * t;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) xv[nt][v] = n < M ? ld_ro_v4(xp + 8 * v) : make_uint4(0u, 0u, 0u, 0u);
+      }
+      uint32_t w[RT][2][B];
+      uint32_t sz[RT][2];
+#pragma unroll
+      for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          lds_unit<B>(st + ((i * RT + rt) * 2 + h) * 8 * kRowG, w[rt][h]);
+          sz[rt][h] = szs[(16 * rt + q + 8 * h) * gmax + gl];
+        }
+      float d[RT][NT][4], dsum[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          dsum[nt][e] = 0.0f;
+#pragma unroll
+          for (int rt = 0; rt < RT; ++rt) d[rt][nt][e] = 0.0f;
+        }
+      uint32_t z2[RT][2];
+      float zf[RT][2];
+      if constexpr (!kFold) {
+#pragma unroll
+        for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t z = sz[rt][h] >> 16;
+            z2[rt][h] = (0x4300u | z) * 0x00010001u;
+            zf[rt][h] = __uint_as_float(0x4B000000u | z);
+          }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint32_t b0[NT], b1[NT];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          b0[nt] = (j & 1) ? xv[nt][j >> 1].z : xv[nt][j >> 1].x;
+          b1[nt] = (j & 1) ? xv[nt][j >> 1].w : xv[nt][j >> 1].y;
+          if constexpr (kFold)
+            mma_bf16_16816(dsum[nt], 0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u, b0[nt], b1[nt]);
+        }
+#pragma unroll
+        for (int rt = 0; rt < RT; ++rt) {
+          uint32_t a0, a1, a2, a3;
+          if constexpr (kFold) {
+            a0 = pair_raw<B>(w[rt][0], 2 * j);
+            a1 = pair_raw<B>(w[rt][1], 2 * j);
+            a2 = pair_raw<B>(w[rt][0], 2 * j + 1);
+            a3 = pair_raw<B>(w[rt][1], 2 * j + 1);
+          } else {
+            a0 = pair_of<B>(w[rt][0], z2[rt][0], zf[rt][0], 2 * j);
+            a1 = pair_of<B>(w[rt][1], z2[rt][1], zf[rt][1], 2 * j);
+            a2 = pair_of<B>(w[rt][0], z2[rt][0], zf[rt][0], 2 * j + 1);
+            a3 = pair_of<B>(w[rt][1], z2[rt][1], zf[rt][1], 2 * j + 1);
+          }
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(d[rt][nt], a0, a1, a2, a3, b0[nt], b1[nt]);
+        }
+      }
+#pragma unroll
+      for (int rt = 0; rt < RT; ++rt) {
+        const float s0 = __half2float(__ushort_as_half(static_cast<uint16_t>(sz[rt][0] & 0xFFFFu)));
+        const float s1 = __half2float(__ushort_as_half(static_cast<uint16_t>(sz[rt][1] & 0xFFFFu)));
+        if constexpr (kFold) {
+          const float zb0 = -static_cast<float>(128u + (sz[rt][0] >> 16));
+          const float zb1 = -static_cast<float>(128u + (sz[rt][1] >> 16));
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            acc[rt][nt][0] = fmaf(s0, fmaf(zb0, dsum[nt][0], d[rt][nt][0]), acc[rt][nt][0]);
+            acc[rt][nt][1] = fmaf(s0, fmaf(zb0, dsum[nt][1], d[rt][nt][1]), acc[rt][nt][1]);
+            acc[rt][nt][2] = fmaf(s1, fmaf(zb1, dsum[nt][2], d[rt][nt][2]), acc[rt][nt][2]);
+            acc[rt][nt][3] = fmaf(s1, fmaf(zb1, dsum[nt][3], d[rt][nt][3]), acc[rt][nt][3]);
+          }
+        } else {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            acc[rt][nt][0] = fmaf(s0, d[rt][nt][0], acc[rt][nt][0]);
+            acc[rt][nt][1] = fmaf(s0, d[rt][nt][1], acc[rt][nt][1]);
+            acc[rt][nt][2] = fmaf(s1, d[rt][nt][2], acc[rt][nt][2]);
+            acc[rt][nt][3] = fmaf(s1, d[rt][nt][3], acc[rt][nt][3]);
+          }
+        }
+      }
+    }
+    __syncwarp();  // the stage is read before the quad may refill it
+  }
+  cp_async_wait<0>();
+  grid_launch_dependents();
+
+  // Add the S warps' partial tiles in warp order (the rings are free now).
+  __syncthreads();
+  float* part = reinterpret_cast<float*>(smem);  // [S][kTile][8 NT + 1]
+  constexpr int kLd = 8 * NT + 1;
+#pragma unroll
+  for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        part[(warp * kTile + 16 * rt + q + 8 * (e >> 1)) * kLd + 8 * nt + 2 * t + (e & 1)] = acc[rt][nt][e];
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < kTile * M; idx += 32 * S) {
+    const int m = idx / kTile, r = idx - m * kTile;
+    const int n = tile0 + r;
+    if (n < N) {
+      float v = part[r * kLd + m];
+#pragma unroll
+      for (int w = 1; w < S; ++w) v += part[(w * kTile + r) * kLd + m];
+      store_y(Y, y_f32, static_cast<int64_t>(m) * N + n, v);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 
@@ -783,6 +1061,103 @@ cudaError_t launch_gemm_decode(const uint16_t* X, int64_t M, int64_t N, int64_t 
     case 6: return launch_b<6>(X, m, n, k, packed, scales, zeros, Y, y_f32, workspace, flags, stream);
     case 7: return launch_b<7>(X, m, n, k, packed, scales, zeros, Y, y_f32, workspace, flags, stream);
     case 8: return launch_b<8>(X, m, n, k, packed, scales, zeros, Y, y_f32, workspace, flags, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+namespace {
+
+template <int B, int RT, int S>
+constexpr int gemv_depth() {  // stages per warp: about 32 KiB of rings per CTA, at least 2
+  constexpr int d = 32 * 1024 / (S * gemv_stage_bytes<B, RT, 2>());
+  return d < 2 ? 2 : d > 8 ? 8 : d;
+}
+
+template <int B, int RT, int S>
+constexpr bool gemv_fits() {  // two stages per warp within 192 KiB
+  return S * 2 * gemv_stage_bytes<B, RT, 2>() <= 192 * 1024;
+}
+
+template <int B, int NT, int RT, int S>
+cudaError_t launch_gemv_cfg(const uint16_t* X, int M, int N, int K, const uint32_t* packed,
+                            const uint16_t* scales, const uint8_t* zeros, void* Y, bool y_f32,
+                            cudaStream_t stream) {
+  constexpr int kGB = 2;
+  constexpr int kD = gemv_depth<B, RT, S>();
+  auto kern = gemm_gemv_kernel<B, NT, RT, S, kGB, kD>;
+  const int G = K / kGroup;
+  const int gmax = (G + S - 1) / S;
+  const size_t rings = static_cast<size_t>(S) * kD * gemv_stage_bytes<B, RT, kGB>();
+  const size_t szb = static_cast<size_t>(S) * 16 * RT * gmax * 4;
+  const size_t partb = static_cast<size_t>(S) * 16 * RT * (8 * NT + 1) * 4;
+  const size_t smem = (rings + szb) > partb ? rings + szb : partb;
+  if (smem > 227 * 1024) return cudaErrorInvalidValue;
+  static int attr_bytes = 0;  // per template instance: the largest size set so far
+  if (static_cast<int>(smem) > attr_bytes) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    attr_bytes = static_cast<int>(smem);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((N + 16 * RT - 1) / (16 * RT)), 1, 1);
+  cfg.blockDim = dim3(32 * S, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, X, M, N, K, reinterpret_cast<const uint8_t*>(packed),
+                            scales, zeros, Y, y_f32 ? 1 : 0, gmax);
+}
+
+template <int B, int NT, int RT>
+cudaError_t launch_gemv_nt(const uint16_t* X, int M, int N, int K, const uint32_t* packed,
+                           const uint16_t* scales, const uint8_t* zeros, void* Y, bool y_f32,
+                           cudaStream_t stream) {
+  // Enough warps to cover the SMs several times over: more K splits for
+  // layers with few row tiles.
+  const int tiles = (N + 16 * RT - 1) / (16 * RT);
+  const int G = K / kGroup;
+  if constexpr (gemv_fits<B, RT, 16>()) {
+    if (tiles < 148 && G >= 16)
+      return launch_gemv_cfg<B, NT, RT, 16>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
+  }
+  if constexpr (gemv_fits<B, RT, 8>()) {
+    if (tiles < 2 * 148 && G >= 8)
+      return launch_gemv_cfg<B, NT, RT, 8>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
+  }
+  return launch_gemv_cfg<B, NT, RT, 4>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
+}
+
+template <int B>
+cudaError_t launch_gemv_b(const uint16_t* X, int M, int N, int K, const uint32_t* packed,
+                          const uint16_t* scales, const uint8_t* zeros, void* Y, bool y_f32,
+                          cudaStream_t stream) {
+  if (M <= 8) return launch_gemv_nt<B, 1, 1>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
+  // Two m16 tiles per warp share each activation fragment; worth it once the
+  // layer has about one 32-row tile per SM.
+  if ((N + 31) / 32 >= 128)
+    return launch_gemv_nt<B, 2, 2>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
+  return launch_gemv_nt<B, 2, 1>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_gemv(const uint16_t* X, int64_t M, int64_t N, int64_t K, int bits,
+                             const uint32_t* packed, const uint16_t* scales, const uint8_t* zeros,
+                             void* Y, bool y_f32, cudaStream_t stream) {
+  const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
+  switch (bits) {
+    case 2: return launch_gemv_b<2>(X, m, n, k, packed, scales, zeros, Y, y_f32, stream);
+    case 3: return launch_gemv_b<3>(X, m, n, k, packed, scales, zeros, Y, y_f32, stream);
+    case 4: return launch_gemv_b<4>(X, m, n, k, packed, scales, zeros, Y, y_f32, stream);
+    case 5: return launch_gemv_b<5>(X, m, n, k, packed, scales, zeros, Y, y_f32, stream);
+    case 6: return launch_gemv_b<6>(X, m, n, k, packed, scales, zeros, Y, y_f32, stream);
+    case 7: return launch_gemv_b<7>(X, m, n, k, packed, scales, zeros, Y, y_f32, stream);
+    case 8: return launch_gemv_b<8>(X, m, n, k, packed, scales, zeros, Y, y_f32, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -37,6 +37,12 @@ cudaError_t launch_gemm_decode(const uint16_t* X, int64_t M, int64_t N, int64_t 
 // device (0 when no row tile is split).
 size_t gemm_decode_workspace_bytes(int64_t N, int64_t K, int bits);
 
+// Split-K GEMV for M <= 16 with no workspace: a CTA per 16-row tile, its
+// warps split K, partial tiles added in shared memory.
+cudaError_t launch_gemm_gemv(const uint16_t* X, int64_t M, int64_t N, int64_t K, int bits,
+                             const uint32_t* packed, const uint16_t* scales, const uint8_t* zeros,
+                             void* Y, bool y_f32, cudaStream_t stream);
+
 // Largest N the decode kernel accepts (the fixed tile-counter region).
 int64_t gemm_decode_max_n();
 

@@ -74,9 +74,9 @@ bool valid_k(int64_t K) { return K >= slq::kGroup && K % slq::kGroup == 0 && K <
 
 bool product_ok(int64_t a, int64_t b) { return a == 0 || b <= kMaxElems / a; }
 
-// Workspace of the kernel `path` selects (only the decode kernel uses one).
+// Workspace of the kernel `path` selects (only the stream-K decode kernel
+// uses one; AUTO never selects it).
 size_t workspace_needed(int64_t M, int64_t N, int64_t K, int bits, slq_gemm_path path) {
-  if (path == SLQ_GEMM_AUTO) path = M <= 16 ? SLQ_GEMM_DECODE : SLQ_GEMM_TILED;
   return (path == SLQ_GEMM_DECODE && M >= 1 && M <= 16 && N >= 1)
              ? slq::gemm_decode_workspace_bytes(N, K, bits)
              : 0;
@@ -95,7 +95,7 @@ slq_status validate_gemm(const void* X, int64_t M, int64_t N, int64_t K, int bit
   if (!aligned(X, 16) || !aligned(packed, 16) || !aligned(Y, 16) || !aligned(scales, 2) ||
       (flags && !aligned(flags, 4)))
     return SLQ_ERR_INVALID_ARGUMENT;
-  if (path != SLQ_GEMM_TILED && M <= 16 && N > slq::gemm_decode_max_n())
+  if (path == SLQ_GEMM_DECODE && N > slq::gemm_decode_max_n())
     return SLQ_ERR_INVALID_ARGUMENT;
   const size_t need = workspace_needed(M, N, K, bits, path);
   if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256)))
@@ -136,7 +136,7 @@ slq_gemm_path slq_gemm_select(int64_t M, int64_t N, int64_t K, int bits) {
   (void)N;
   (void)K;
   (void)bits;
-  return M <= 16 ? SLQ_GEMM_DECODE : SLQ_GEMM_TILED;
+  return M <= 16 ? SLQ_GEMM_GEMV : SLQ_GEMM_TILED;
 }
 
 slq_status slq_quantize(const void* W_bf16, int64_t N, int64_t K, int bits, uint32_t* packed,
@@ -164,16 +164,17 @@ size_t slq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits) {
   if (M < 0 || N < 0 || M > kMaxDim || N > kMaxDim || !valid_k(K) || !valid_bits(bits) ||
       !product_ok(N, K))
     return 0;
-  return workspace_needed(M, N, K, bits, SLQ_GEMM_AUTO);
+  return M <= 16 ? workspace_needed(M, N, K, bits, SLQ_GEMM_DECODE) : 0;
 }
 
 slq_status slq_gemm_ex(const void* X_bf16, int64_t M, int64_t N, int64_t K, int bits,
                        const uint32_t* packed, const void* scales_f16, const uint8_t* zeros,
                        void* Y, slq_dtype y_dtype, slq_gemm_path path, void* workspace,
                        size_t workspace_bytes, uint32_t* flags, void* stream) {
-  if (path != SLQ_GEMM_AUTO && path != SLQ_GEMM_DECODE && path != SLQ_GEMM_TILED)
+  if (path != SLQ_GEMM_AUTO && path != SLQ_GEMM_DECODE && path != SLQ_GEMM_TILED &&
+      path != SLQ_GEMM_GEMV)
     return SLQ_ERR_INVALID_ARGUMENT;
-  if (path == SLQ_GEMM_DECODE && M > 16) return SLQ_ERR_INVALID_ARGUMENT;
+  if ((path == SLQ_GEMM_DECODE || path == SLQ_GEMM_GEMV) && M > 16) return SLQ_ERR_INVALID_ARGUMENT;
   const slq_status v = validate_gemm(X_bf16, M, N, K, bits, packed, scales_f16, zeros, Y, y_dtype,
                                      path, workspace, workspace_bytes, flags);
   if (v != SLQ_OK) return v;
@@ -185,6 +186,8 @@ slq_status slq_gemm_ex(const void* X_bf16, int64_t M, int64_t N, int64_t K, int 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const uint16_t* X = static_cast<const uint16_t*>(X_bf16);
   const uint16_t* sc = static_cast<const uint16_t*>(scales_f16);
+  if (path == SLQ_GEMM_GEMV)
+    return from_cuda(slq::launch_gemm_gemv(X, M, N, K, bits, packed, sc, zeros, Y, f32, s));
   if (path == SLQ_GEMM_DECODE)
     return from_cuda(
         slq::launch_gemm_decode(X, M, N, K, bits, packed, sc, zeros, Y, f32, workspace, flags, s));
