@@ -22,8 +22,9 @@ pages' models (no checkpoints or datasets here).
 timed ones) and prints {"case", "avg_us", ...}: the command the profiles'
 ncu captures use.  SPEC is one of
   block                     the 21 decode launches of the Qwen3-8B block
-  decode:N:K:b:M            one decode-path dequant-GEMM
-  tiled:N:K:b:M             one tiled-path dequant-GEMM
+  gemv:N:K:b:M              one dequant-GEMM on the split-K GEMV kernel (M <= 16)
+  decode:N:K:b:M            one dequant-GEMM on the stream-K decode kernel (M <= 16)
+  tiled:N:K:b:M             one dequant-GEMM on the tiled tcgen05 kernel
   ear:T:V:tau               one EAR/KL reduction
   quantize:N:K:b            one quantize+pack
 
@@ -606,7 +607,7 @@ def run_case(args):
             for x, qw, y in items:
                 slq.gemm(x, qw, out=y, stream=stream)
         per_call = len(items)
-    elif kind in ("decode", "tiled"):
+    elif kind in ("gemv", "decode", "tiled"):
         N, K, b, M = vals
         qw = slq.quantize(synth.weights_torch(N, K, device=dev), b)
         x = synth.activations_torch(M, K, device=dev)

@@ -804,6 +804,114 @@ __global__ void __launch_bounds__(32 * S)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[rt][nt][e] = 0.0f;
 
+  // Activation fragments X[n][128 g + 32 t + 4 j .. + 3] (k-step j) of one
+  // group; loaded one group ahead, alternating between two register sets.
+  auto load_x = [&](int g, uint4 (&xv)[NT][4]) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int n = q + 8 * nt;
+      const uint16_t* xp = X + static_cast<int64_t>(n) * K + g * kGroup + 32 * t;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) xv[nt][v] = n < M ? ld_ro_v4(xp + 8 * v) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  auto group = [&](const uint8_t* st, int i, int gl, const uint4 (&xpre)[NT][4]) {
+    // M <= 8: the fragments came one group ahead; M > 8: loaded here (two
+    // register sets of 32 would spill next to two row tiles).
+    uint4 xj[NT][4];
+    if constexpr (NT == 2) load_x(g0 + gl, xj);
+    const uint4(*xv)[4] = (NT == 2) ? xj : xpre;
+    uint32_t w[RT][2][B];
+    uint32_t sz[RT][2];
+#pragma unroll
+    for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        lds_unit<B>(st + ((i * RT + rt) * 2 + h) * 8 * kRowG, w[rt][h]);
+        sz[rt][h] = szs[(16 * rt + q + 8 * h) * gmax + gl];
+      }
+    float d[RT][NT][4], dsum[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        dsum[nt][e] = 0.0f;
+#pragma unroll
+        for (int rt = 0; rt < RT; ++rt) d[rt][nt][e] = 0.0f;
+      }
+    uint32_t z2[RT][2];
+    float zf[RT][2];
+    if constexpr (!kFold) {
+#pragma unroll
+      for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t z = sz[rt][h] >> 16;
+          z2[rt][h] = (0x4300u | z) * 0x00010001u;
+          zf[rt][h] = __uint_as_float(0x4B000000u | z);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      uint32_t b0[NT], b1[NT];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        b0[nt] = (j & 1) ? xv[nt][j >> 1].z : xv[nt][j >> 1].x;
+        b1[nt] = (j & 1) ? xv[nt][j >> 1].w : xv[nt][j >> 1].y;
+        if constexpr (kFold)
+          mma_bf16_16816(dsum[nt], 0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u, b0[nt], b1[nt]);
+      }
+#pragma unroll
+      for (int rt = 0; rt < RT; ++rt) {
+        uint32_t a0, a1, a2, a3;
+        if constexpr (kFold) {
+          a0 = pair_raw<B>(w[rt][0], 2 * j);
+          a1 = pair_raw<B>(w[rt][1], 2 * j);
+          a2 = pair_raw<B>(w[rt][0], 2 * j + 1);
+          a3 = pair_raw<B>(w[rt][1], 2 * j + 1);
+        } else {
+          a0 = pair_of<B>(w[rt][0], z2[rt][0], zf[rt][0], 2 * j);
+          a1 = pair_of<B>(w[rt][1], z2[rt][1], zf[rt][1], 2 * j);
+          a2 = pair_of<B>(w[rt][0], z2[rt][0], zf[rt][0], 2 * j + 1);
+          a3 = pair_of<B>(w[rt][1], z2[rt][1], zf[rt][1], 2 * j + 1);
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(d[rt][nt], a0, a1, a2, a3, b0[nt], b1[nt]);
+      }
+    }
+#pragma unroll
+    for (int rt = 0; rt < RT; ++rt) {
+      const float s0 = __half2float(__ushort_as_half(static_cast<uint16_t>(sz[rt][0] & 0xFFFFu)));
+      const float s1 = __half2float(__ushort_as_half(static_cast<uint16_t>(sz[rt][1] & 0xFFFFu)));
+      if constexpr (kFold) {
+        const float zb0 = -static_cast<float>(128u + (sz[rt][0] >> 16));
+        const float zb1 = -static_cast<float>(128u + (sz[rt][1] >> 16));
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          acc[rt][nt][0] = fmaf(s0, fmaf(zb0, dsum[nt][0], d[rt][nt][0]), acc[rt][nt][0]);
+          acc[rt][nt][1] = fmaf(s0, fmaf(zb0, dsum[nt][1], d[rt][nt][1]), acc[rt][nt][1]);
+          acc[rt][nt][2] = fmaf(s1, fmaf(zb1, dsum[nt][2], d[rt][nt][2]), acc[rt][nt][2]);
+          acc[rt][nt][3] = fmaf(s1, fmaf(zb1, dsum[nt][3], d[rt][nt][3]), acc[rt][nt][3]);
+        }
+      } else {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          acc[rt][nt][0] = fmaf(s0, d[rt][nt][0], acc[rt][nt][0]);
+          acc[rt][nt][1] = fmaf(s0, d[rt][nt][1], acc[rt][nt][1]);
+          acc[rt][nt][2] = fmaf(s1, d[rt][nt][2], acc[rt][nt][2]);
+          acc[rt][nt][3] = fmaf(s1, d[rt][nt][3], acc[rt][nt][3]);
+        }
+      }
+    }
+  };
+
+  // Two groups per stage (GB = 2): for M <= 8 the first computes from xa
+  // while xb is loaded for the second, which loads xa for the next stage's
+  // first.
+  static_assert(GB == 2, "the activation double buffer alternates within a stage");
+  constexpr bool kAhead = NT == 1;
+  uint4 xa[NT][4], xb[NT][4];
+  if (kAhead && ng > 0) load_x(g0, xa);
   for (int bi = 0; bi < nb; ++bi) {
     const int nx = bi + D - 1;
     if (nx < nb) issue(nx % D, g0 + nx * GB);
@@ -811,102 +919,12 @@ __global__ void __launch_bounds__(32 * S)
     cp_async_wait<D - 1>();
     __syncwarp();  // the quad's chunks of every row are in
     const uint8_t* st = ring + (bi % D) * kStage + q * kRowG + 4 * B * t;
-#pragma unroll
-    for (int i = 0; i < GB; ++i) {
-      const int gl = bi * GB + i;  // group index within this warp's range
-      if (gl >= ng) break;
-      const int g = g0 + gl;
-      // Activation fragments: X[n][128 g + 32 t + 4 j .. + 3] for k-step j.
-      uint4 xv[NT][4];
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int n = q + 8 * nt;
-        const uint16_t* xp = X + static_cast<int64_t>(n) * K + g * kGroup + 32 * t;
-#pragma unroll
-        for (int v = 0; v < 4; ++v) xv[nt][v] = n < M ? ld_ro_v4(xp + 8 * v) : make_uint4(0u, 0u, 0u, 0u);
-      }
-      uint32_t w[RT][2][B];
-      uint32_t sz[RT][2];
-#pragma unroll
-      for (int rt = 0; rt < RT; ++rt)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          lds_unit<B>(st + ((i * RT + rt) * 2 + h) * 8 * kRowG, w[rt][h]);
-          sz[rt][h] = szs[(16 * rt + q + 8 * h) * gmax + gl];
-        }
-      float d[RT][NT][4], dsum[NT][4];
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          dsum[nt][e] = 0.0f;
-#pragma unroll
-          for (int rt = 0; rt < RT; ++rt) d[rt][nt][e] = 0.0f;
-        }
-      uint32_t z2[RT][2];
-      float zf[RT][2];
-      if constexpr (!kFold) {
-#pragma unroll
-        for (int rt = 0; rt < RT; ++rt)
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t z = sz[rt][h] >> 16;
-            z2[rt][h] = (0x4300u | z) * 0x00010001u;
-            zf[rt][h] = __uint_as_float(0x4B000000u | z);
-          }
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        uint32_t b0[NT], b1[NT];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          b0[nt] = (j & 1) ? xv[nt][j >> 1].z : xv[nt][j >> 1].x;
-          b1[nt] = (j & 1) ? xv[nt][j >> 1].w : xv[nt][j >> 1].y;
-          if constexpr (kFold)
-            mma_bf16_16816(dsum[nt], 0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u, b0[nt], b1[nt]);
-        }
-#pragma unroll
-        for (int rt = 0; rt < RT; ++rt) {
-          uint32_t a0, a1, a2, a3;
-          if constexpr (kFold) {
-            a0 = pair_raw<B>(w[rt][0], 2 * j);
-            a1 = pair_raw<B>(w[rt][1], 2 * j);
-            a2 = pair_raw<B>(w[rt][0], 2 * j + 1);
-            a3 = pair_raw<B>(w[rt][1], 2 * j + 1);
-          } else {
-            a0 = pair_of<B>(w[rt][0], z2[rt][0], zf[rt][0], 2 * j);
-            a1 = pair_of<B>(w[rt][1], z2[rt][1], zf[rt][1], 2 * j);
-            a2 = pair_of<B>(w[rt][0], z2[rt][0], zf[rt][0], 2 * j + 1);
-            a3 = pair_of<B>(w[rt][1], z2[rt][1], zf[rt][1], 2 * j + 1);
-          }
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(d[rt][nt], a0, a1, a2, a3, b0[nt], b1[nt]);
-        }
-      }
-#pragma unroll
-      for (int rt = 0; rt < RT; ++rt) {
-        const float s0 = __half2float(__ushort_as_half(static_cast<uint16_t>(sz[rt][0] & 0xFFFFu)));
-        const float s1 = __half2float(__ushort_as_half(static_cast<uint16_t>(sz[rt][1] & 0xFFFFu)));
-        if constexpr (kFold) {
-          const float zb0 = -static_cast<float>(128u + (sz[rt][0] >> 16));
-          const float zb1 = -static_cast<float>(128u + (sz[rt][1] >> 16));
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            acc[rt][nt][0] = fmaf(s0, fmaf(zb0, dsum[nt][0], d[rt][nt][0]), acc[rt][nt][0]);
-            acc[rt][nt][1] = fmaf(s0, fmaf(zb0, dsum[nt][1], d[rt][nt][1]), acc[rt][nt][1]);
-            acc[rt][nt][2] = fmaf(s1, fmaf(zb1, dsum[nt][2], d[rt][nt][2]), acc[rt][nt][2]);
-            acc[rt][nt][3] = fmaf(s1, fmaf(zb1, dsum[nt][3], d[rt][nt][3]), acc[rt][nt][3]);
-          }
-        } else {
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            acc[rt][nt][0] = fmaf(s0, d[rt][nt][0], acc[rt][nt][0]);
-            acc[rt][nt][1] = fmaf(s0, d[rt][nt][1], acc[rt][nt][1]);
-            acc[rt][nt][2] = fmaf(s1, d[rt][nt][2], acc[rt][nt][2]);
-            acc[rt][nt][3] = fmaf(s1, d[rt][nt][3], acc[rt][nt][3]);
-          }
-        }
-      }
+    const int gl = bi * GB;
+    if (kAhead && gl + 1 < ng) load_x(g0 + gl + 1, xb);
+    group(st, 0, gl, xa);
+    if (gl + 1 < ng) {
+      if (kAhead && gl + 2 < ng) load_x(g0 + gl + 2, xa);
+      group(st, 1, gl + 1, xb);
     }
     __syncwarp();  // the stage is read before the quad may refill it
   }
@@ -1068,14 +1086,14 @@ cudaError_t launch_gemm_decode(const uint16_t* X, int64_t M, int64_t N, int64_t 
 namespace {
 
 template <int B, int RT, int S>
-constexpr int gemv_depth() {  // stages per warp: about 32 KiB of rings per CTA, at least 2
-  constexpr int d = 32 * 1024 / (S * gemv_stage_bytes<B, RT, 2>());
+constexpr int gemv_depth() {  // stages per warp: about 6 KiB of ring per warp, 2..8
+  constexpr int d = 6 * 1024 / gemv_stage_bytes<B, RT, 2>();
   return d < 2 ? 2 : d > 8 ? 8 : d;
 }
 
 template <int B, int RT, int S>
-constexpr bool gemv_fits() {  // two stages per warp within 192 KiB
-  return S * 2 * gemv_stage_bytes<B, RT, 2>() <= 192 * 1024;
+constexpr bool gemv_fits() {  // the CTA's rings within 192 KiB
+  return S * gemv_depth<B, RT, S>() * gemv_stage_bytes<B, RT, 2>() <= 192 * 1024;
 }
 
 template <int B, int NT, int RT, int S>
@@ -1117,16 +1135,17 @@ template <int B, int NT, int RT>
 cudaError_t launch_gemv_nt(const uint16_t* X, int M, int N, int K, const uint32_t* packed,
                            const uint16_t* scales, const uint8_t* zeros, void* Y, bool y_f32,
                            cudaStream_t stream) {
-  // Enough warps to cover the SMs several times over: more K splits for
-  // layers with few row tiles.
+  // K splits per row tile: 4 warps per tile once the layer has about 16
+  // warps' worth of 16-row blocks per SM, more splits for layers with fewer
+  // (measured on this B200 over the Qwen3-8B and 8192 x 8192 layers).
   const int tiles = (N + 16 * RT - 1) / (16 * RT);
   const int G = K / kGroup;
   if constexpr (gemv_fits<B, RT, 16>()) {
-    if (tiles < 148 && G >= 16)
+    if (tiles < 148 && G >= 32)
       return launch_gemv_cfg<B, NT, RT, 16>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
   }
   if constexpr (gemv_fits<B, RT, 8>()) {
-    if (tiles < 2 * 148 && G >= 8)
+    if (tiles * RT < 600 && G >= 16)
       return launch_gemv_cfg<B, NT, RT, 8>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
   }
   return launch_gemv_cfg<B, NT, RT, 4>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
