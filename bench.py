@@ -566,10 +566,10 @@ def run_reference(args, rank, world):
 
 def decode_traffic():
     """DRAM bytes per decode launch of this workload from the committed ncu
-    capture (profiles/decode_block_traffic.json), or None when the kernel
+    capture (profiles/decode_block_traffic.txt), or None when the kernel
     source has changed since it was taken."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "decode_block_traffic.json")
+    path = os.path.join(ROOT, "profiles", "decode_block_traffic.txt")
     src = os.path.join(ROOT, "weight_only_mixed_b200", "csrc", "gemm_decode.cu")
     try:
         with open(path) as f:
