@@ -217,20 +217,29 @@ def run_slq(args, rank, world, local_rank):
             ev.record(k, sh)
 
     # Warm up eagerly once (device attributes, first launches), then capture.
+    # The timed graphs hold only the kernels, so consecutive launches overlap
+    # (programmatic dependent launch); a second set with an event between
+    # kernels gives the per-launch durations and is replayed after the timed
+    # region.
     step_body(0)
     torch.cuda.synchronize()
-    graphs = []
+    graphs, ev_graphs = [], []
     for r in range(R):
         g = torch.cuda.CUDAGraph()
-        try:
-            with torch.cuda.graph(g, stream=stream):
-                step_body(r, gev[r] if gev else None)
-        except Exception:
-            gev = None
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                step_body(r)
+        with torch.cuda.graph(g, stream=stream):
+            step_body(r)
         graphs.append(g)
+        if gev is not None:
+            ge = torch.cuda.CUDAGraph()
+            try:
+                with torch.cuda.graph(ge, stream=stream):
+                    step_body(r, gev[r])
+                ev_graphs.append(ge)
+            except Exception:
+                gev = None
+    torch.cuda.synchronize()
+    for g in graphs:  # first replay uploads the graph
+        g.replay()
     torch.cuda.synchronize()
 
     dist = None
@@ -266,11 +275,14 @@ def run_slq(args, rank, world, local_rank):
 
     value = world * 3 * BLOCK_BYTES / (ms_step * 1e-3) / 1e9  # GB/s, whole job
 
-    # Per-launch durations of the decode kernel from the last replay of each
-    # graph inside the timed region.
+    # Per-launch durations of the decode kernel: one replay of each
+    # event-instrumented graph after the timed region.
     per_m = {}
     kernel_ms = None
-    if gev is not None and args.steps * reps >= R:
+    if gev is not None and len(ev_graphs) == R:
+        for ge in ev_graphs:
+            ge.replay()
+        torch.cuda.synchronize()
         tot_bytes, tot_ms = 0.0, 0.0
         for r in range(R):
             k = 0
@@ -332,7 +344,7 @@ def run_slq(args, rank, world, local_rank):
         rows = other_rows(args, slq, synth, torch, dev, stream, hbm_peak, tc_peak, rank)
 
     # free the rotated copies before the CPU baseline
-    del layers, graphs
+    del layers, graphs, ev_graphs
     torch.cuda.synchronize()
 
     out = None

@@ -24,11 +24,12 @@ namespace slq {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
-// Ring kernel shape: 16 consumer warps, two 16-byte units of each logit
-// stream per consumer thread per stage (a 32 KiB stage), six stages.
+// Ring kernel shape: 16 consumer warps, three 16-byte units of each logit
+// stream per consumer thread per stage (a 48 KiB stage), four stages
+// (measured against 12-24 warps and 2-3 units on T = 4096, V = 151936).
 constexpr int kEarConsumerWarps = 16;
-constexpr int kEarUnits = 2;
-constexpr int kEarStages = 6;
+constexpr int kEarUnits = 3;
+constexpr int kEarStages = 4;
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
