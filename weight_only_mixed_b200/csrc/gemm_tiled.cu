@@ -453,13 +453,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t base = tmem + (static_cast<uint32_t>(32 * q) << 16) +
                               static_cast<uint32_t>(buf * kChains * BN + hcol * kHalf);
         if constexpr (kHalf % 16 == 0) {
+          // Four column blocks of 16 per TMEM wait (the wait covers every
+          // load issued before it): one wait per block left the fold
+          // latency-bound, about 10 % of the kernel's time at M >= 1024.
+          constexpr int kPer = (kHalf / 16) % 4 == 0 ? 4 : 1;
 #pragma unroll
-          for (int c = 0; c < kHalf / 16; ++c) {
-            uint32_t r[16];
-            tmem_ld_32x32b_x16(base + 16 * c, r);
+          for (int c = 0; c < kHalf / 16; c += kPer) {
+            uint32_t r[kPer][16];
+#pragma unroll
+            for (int e = 0; e < kPer; ++e) tmem_ld_32x32b_x16(base + 16 * (c + e), r[e]);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) acc[16 * c + i] = fmaf(s, __uint_as_float(r[i]), acc[16 * c + i]);
+            for (int e = 0; e < kPer; ++e)
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                acc[16 * (c + e) + i] = fmaf(s, __uint_as_float(r[e][i]), acc[16 * (c + e) + i]);
           }
         } else {
           // Decode tile: sum the kChains partial accumulators in a fixed order.
