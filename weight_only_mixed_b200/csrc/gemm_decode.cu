@@ -1155,7 +1155,16 @@ template <int B>
 cudaError_t launch_gemv_b(const uint16_t* X, int M, int N, int K, const uint32_t* packed,
                           const uint16_t* scales, const uint8_t* zeros, void* Y, bool y_f32,
                           cudaStream_t stream) {
-  if (M <= 8) return launch_gemv_nt<B, 1, 1>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
+  if (M <= 8) {
+    // Two m16 tiles per warp also pay at M <= 8 for b <= 6, where the
+    // per-group activation and scale work is a larger share (measured; at
+    // b = 7, 8 the doubled unit registers cost more than they save).
+    if constexpr (B <= 6) {
+      if ((N + 31) / 32 >= 128)
+        return launch_gemv_nt<B, 1, 2>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
+    }
+    return launch_gemv_nt<B, 1, 1>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
+  }
   // Two m16 tiles per warp share each activation fragment; worth it once the
   // layer has about one 32-row tile per SM.
   if ((N + 31) / 32 >= 128)
