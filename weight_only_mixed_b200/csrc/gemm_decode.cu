@@ -1141,7 +1141,7 @@ cudaError_t launch_gemv_nt(const uint16_t* X, int M, int N, int K, const uint32_
   const int tiles = (N + 16 * RT - 1) / (16 * RT);
   const int G = K / kGroup;
   if constexpr (gemv_fits<B, RT, 16>()) {
-    if (tiles < 148 && G >= 32)
+    if ((NT == 2 ? tiles : tiles * RT) < 148 && G >= 32)
       return launch_gemv_cfg<B, NT, RT, 16>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
   }
   if constexpr (gemv_fits<B, RT, 8>()) {
