@@ -5,7 +5,9 @@ Headline workload: a Qwen3-8B-shaped decoder block at decode batch sizes --
 hidden 4096, q/o 4096x4096 at 5 bits, k/v 1024x4096 at 8 bits, gate/up
 12288x4096 and down 4096x12288 at 4 bits (asymmetric INT, group 128), X bf16
 ~ N(0,1) at M in {1, 4, 16}.  One step = the 7 dequantize-GEMMs of the block
-at each of the three M (21 launches, replayed as one CUDA graph).  The metric
+at each of the three M, replayed as one CUDA graph; the projections that read
+the same input in a decoder block run as one slq_gemm_group launch (q+k+v,
+gate+up), so a step is 12 launches.  The metric
 is packed-weight bytes streamed per second (codes + fp16 scales + uint8
 zeros), whole job over all ranks.
 
@@ -21,7 +23,7 @@ pages' models (no checkpoints or datasets here).
 --case runs one kernel of the path on its own (W untimed launches, then K
 timed ones) and prints {"case", "avg_us", ...}: the command the profiles'
 ncu captures use.  SPEC is one of
-  block                     the 21 decode launches of the Qwen3-8B block
+  block                     the 12 decode launches of one Qwen3-8B block step
   gemv:N:K:b:M              one dequant-GEMM on the split-K GEMV kernel (M <= 16)
   decode:N:K:b:M            one dequant-GEMM on the stream-K decode kernel (M <= 16)
   tiled:N:K:b:M             one dequant-GEMM on the tiled tcgen05 kernel
@@ -58,6 +60,9 @@ QWEN3_8B_BLOCK = [("q", 4096, 4096, 5), ("k", 1024, 4096, 8), ("v", 1024, 4096, 
                   ("o", 4096, 4096, 5), ("gate", 12288, 4096, 4), ("up", 12288, 4096, 4),
                   ("down", 4096, 12288, 4)]
 DECODE_MS = (1, 4, 16)
+# Launches of one block at one M: the projections that read the same input
+# in a decoder block run as one grouped launch (q, k, v; gate, up).
+BLOCK_LAUNCHES = ((0, 1, 2), (3,), (4, 5), (6,))
 METRIC = "W{2-8}A16 GEMM weight GB/s (% HBM peak) & TFLOP/s per b and M; EAR/KL GB/s"
 
 
@@ -199,7 +204,16 @@ def run_slq(args, rank, world, local_rank):
              for (_, N, K, b) in QWEN3_8B_BLOCK] for M in DECODE_MS}
     torch.cuda.synchronize()
 
-    n_launch = len(DECODE_MS) * len(QWEN3_8B_BLOCK)
+    n_launch = len(DECODE_MS) * len(BLOCK_LAUNCHES)
+
+    def block_launch(M, r, grp, xs=None):
+        xs = xs if xs is not None else X[M]
+        if len(grp) == 1:
+            i = grp[0]
+            slq.gemm(xs[i], layers[r][i], out=Y[M][i], stream=stream)
+        else:
+            slq.gemm_group([(xs[i], layers[r][i]) for i in grp], outs=[Y[M][i] for i in grp],
+                           stream=stream)
     try:
         gev = [GraphEvents(n_launch + 1) for _ in range(R)]
     except Exception:
@@ -208,10 +222,10 @@ def run_slq(args, rank, world, local_rank):
     def step_body(r, ev=None):
         k = 0
         for M in DECODE_MS:
-            for i in range(len(QWEN3_8B_BLOCK)):
+            for grp in BLOCK_LAUNCHES:
                 if ev is not None:
                     ev.record(k, sh)
-                slq.gemm(X[M][i], layers[r][i], out=Y[M][i], stream=stream)
+                block_launch(M, r, grp)
                 k += 1
         if ev is not None:
             ev.record(k, sh)
@@ -287,9 +301,9 @@ def run_slq(args, rank, world, local_rank):
         for r in range(R):
             k = 0
             for M in DECODE_MS:
-                for i, (name, N, K, b) in enumerate(QWEN3_8B_BLOCK):
+                for grp in BLOCK_LAUNCHES:
                     d = gev[r].elapsed_ms(k, k + 1)
-                    wb = weight_bytes(N, K, b)
+                    wb = sum(weight_bytes(*QWEN3_8B_BLOCK[i][1:]) for i in grp)
                     per_m.setdefault(M, [0.0, 0.0])
                     per_m[M][0] += wb
                     per_m[M][1] += d
@@ -313,10 +327,12 @@ def run_slq(args, rank, world, local_rank):
 
     def e2e_step(r):
         for M in DECODE_MS:
-            for i in range(len(QWEN3_8B_BLOCK)):
-                Xd[M][i].copy_(Xh[M][i], non_blocking=True)
-                slq.gemm(Xd[M][i], layers[r][i], out=Y[M][i], stream=stream)
-                Yh[M][i].copy_(Y[M][i], non_blocking=True)
+            for grp in BLOCK_LAUNCHES:
+                for i in grp:
+                    Xd[M][i].copy_(Xh[M][i], non_blocking=True)
+                block_launch(M, r, grp, Xd[M])
+                for i in grp:
+                    Yh[M][i].copy_(Y[M][i], non_blocking=True)
         stream.synchronize()
 
     for s in range(max(1, args.warmup)):
@@ -366,7 +382,8 @@ def run_slq(args, rank, world, local_rank):
             "config": {
                 "workload": "Qwen3-8B-shaped decoder block decode: q/o 4096x4096 b5, k/v 1024x4096 b8, "
                             "gate/up 12288x4096 b4, down 4096x12288 b4, asymmetric INT g128; "
-                            "M in {1,4,16}; 21 dequant-GEMM launches per step (one CUDA graph)",
+                            "M in {1,4,16}; per M: q+k+v in one slq_gemm_group launch, o, gate+up in one, down "
+                            "(12 launches per step, one CUDA graph); independent X per projection",
                 "block_weight_bytes": BLOCK_BYTES,
                 "bytes_per_step": 3 * BLOCK_BYTES,
                 "l2": f"inputs larger than L2: {R} rotated weight copies ({R * BLOCK_BYTES / 2**20:.0f} MiB > 126 MiB L2)",
@@ -607,18 +624,22 @@ def run_case(args):
     kind, *parts = args.case.split(":")
     vals = [float(p) if "." in p else int(p) for p in parts]
     if kind == "block":
-        items = []
+        calls = []
         for M in DECODE_MS:
-            for i, (_, N, K, b) in enumerate(QWEN3_8B_BLOCK):
-                qw = slq.quantize(synth.weights_torch(N, K, seed=synth.SEED_WEIGHTS + 10 * i, device=dev), b)
-                x = synth.activations_torch(M, K, seed=synth.SEED_X + 10 * i + M, device=dev)
-                y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-                items.append((x, qw, y))
+            qws = [slq.quantize(synth.weights_torch(N, K, seed=synth.SEED_WEIGHTS + 10 * i, device=dev), b)
+                   for i, (_, N, K, b) in enumerate(QWEN3_8B_BLOCK)]
+            xs = [synth.activations_torch(M, K, seed=synth.SEED_X + 10 * i + M, device=dev)
+                  for i, (_, N, K, b) in enumerate(QWEN3_8B_BLOCK)]
+            for grp in BLOCK_LAUNCHES:
+                calls.append([(xs[i], qws[i]) for i in grp])
 
         def fn():
-            for x, qw, y in items:
-                slq.gemm(x, qw, out=y, stream=stream)
-        per_call = len(items)
+            for items in calls:
+                if len(items) == 1:
+                    slq.gemm(items[0][0], items[0][1], stream=stream)
+                else:
+                    slq.gemm_group(items, stream=stream)
+        per_call = len(calls)
     elif kind in ("gemv", "decode", "tiled"):
         N, K, b, M = vals
         qw = slq.quantize(synth.weights_torch(N, K, device=dev), b)

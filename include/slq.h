@@ -181,6 +181,45 @@ slq_status slq_gemm_ex(const void *X_bf16, int64_t M, int64_t N, int64_t K,
                        slq_dtype y_dtype, slq_gemm_path path, void *workspace,
                        size_t workspace_bytes, uint32_t *flags, void *stream);
 
+/* One layer of slq_gemm_group: Y = X W^T with the arguments of slq_gemm. */
+typedef struct {
+  const void *X_bf16;        /* [M, K] bf16, device */
+  int64_t N, K;              /* N >= 0 (0: the layer is skipped), K >= 128, K % 128 == 0 */
+  int bits;                  /* 2..8 */
+  const uint32_t *packed;    /* as written by slq_quantize */
+  const void *scales_f16;
+  const uint8_t *zeros;
+  void *Y;                   /* [M, N] of the call's y_dtype, device, written */
+} slq_gemm_layer;
+
+/*
+ * slq_gemm_group -- several decode-step layers in ONE launch of the
+ * SLQ_GEMM_GEMV kernel: for each layer i, Y_i = X_i W_i^T.
+ *
+ * Source: the pages serve every linear layer of a block at its own bitwidth
+ * (GitHub README, "4. Build and serve a checkpoint"; gist.science summary,
+ * Key Results "Inference Speedup").  The projections that read the same
+ * input in a decoder block (q, k, v; gate, up) can run as one launch even
+ * when their b differ, which removes the per-launch start and tail costs
+ * that dominate decode-sized layers.
+ *
+ * layers      host array of `count` slq_gemm_layer; any mix of b, N and K.
+ * count       1 .. slq_gemm_group_max().
+ * M           0..16 (0 launches nothing), shared by the layers.
+ * y_dtype, flags, stream   as for slq_gemm.
+ *
+ * Each Y_i meets slq_gemm's tolerance, and repeated calls with the same
+ * layers give identical bits; the order of the K-split sum follows the
+ * group's size, so Y_i may differ in the last bits from a single-layer call.
+ * No output may overlap any layer's inputs or another output
+ * (SLQ_ERR_INVALID_ARGUMENT); every layer is validated as in slq_gemm.
+ */
+slq_status slq_gemm_group(const slq_gemm_layer *layers, int count, int64_t M,
+                          slq_dtype y_dtype, uint32_t *flags, void *stream);
+
+/* Most layers slq_gemm_group takes in one call (8). */
+int slq_gemm_group_max(void);
+
 /*
  * slq_gemm_decode_static -- slq_gemm for decode batches (M <= 16) that
  * allocates nothing and takes no workspace.

@@ -139,3 +139,37 @@ def test_valid_calls_without_a_device_are_refused():
     assert _q() == slq.SLQ_ERR_UNSUPPORTED_DEVICE
     assert _g() == slq.SLQ_ERR_UNSUPPORTED_DEVICE
     assert _e() == slq.SLQ_ERR_UNSUPPORTED_DEVICE
+
+
+def _layer(X=FAKE, N=8, K=256, bits=4, off=0):
+    base = FAKE + ((1 + 8 * off) << 24)
+    return slq.GemmLayer(X, N, K, bits, base, base + (1 << 24), base + (2 << 24), base + (3 << 24))
+
+
+def _grp(layers, M=4, dtype=0, flags=None):
+    arr = (slq.GemmLayer * max(1, len(layers)))(*layers)
+    return L.slq_gemm_group(arr if layers else None, len(layers), M, dtype, flags, None)
+
+
+def test_gemm_group_validation():
+    assert L.slq_gemm_group_max() == 8
+    ok = [_layer(off=0), _layer(X=FAKE + (100 << 24), N=16, K=512, bits=7, off=1)]
+    # Valid arguments reach the device check (no GPU here) or run.
+    assert _grp(ok) in (slq.SLQ_OK, slq.SLQ_ERR_UNSUPPORTED_DEVICE)
+    assert _grp(ok, M=0) == slq.SLQ_OK
+    bad = [
+        _grp([]),                                               # no layers
+        _grp([_layer(off=i) for i in range(9)]),                # more than 8
+        _grp(ok, M=17),                                         # decode sizes only
+        _grp(ok, dtype=2),
+        _grp([_layer(K=100)]),                                  # K % 128
+        _grp([_layer(bits=9)]),
+        _grp([_layer(X=FAKE + 8)]),                             # misaligned X
+        # layer 1's Y lands on layer 0's packed weights
+        _grp([_layer(off=0), slq.GemmLayer(FAKE + (100 << 24), 8, 256, 4, FAKE + (9 << 24),
+                                           FAKE + (10 << 24), FAKE + (11 << 24), FAKE + (1 << 24))]),
+        # two layers write the same Y
+        _grp([_layer(off=0), slq.GemmLayer(FAKE + (100 << 24), 8, 256, 4, FAKE + (9 << 24),
+                                           FAKE + (10 << 24), FAKE + (11 << 24), FAKE + (4 << 24))]),
+    ]
+    assert all(r == slq.SLQ_ERR_INVALID_ARGUMENT for r in bad), bad

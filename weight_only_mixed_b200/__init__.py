@@ -80,6 +80,18 @@ _lib.slq_ear_kl.argtypes = [_P, _P, _I64, _I64, ctypes.c_float, _P, _P, _P, _P, 
 _lib.slq_ear_kl.restype = _I
 
 
+class GemmLayer(ctypes.Structure):
+    """slq_gemm_layer: one layer of slq_gemm_group."""
+    _fields_ = [("X_bf16", _P), ("N", _I64), ("K", _I64), ("bits", _I), ("packed", _P),
+                ("scales_f16", _P), ("zeros", _P), ("Y", _P)]
+
+
+_lib.slq_gemm_group.argtypes = [ctypes.POINTER(GemmLayer), _I, _I64, _I, _P, _P]
+_lib.slq_gemm_group.restype = _I
+_lib.slq_gemm_group_max.argtypes = []
+_lib.slq_gemm_group_max.restype = _I
+
+
 def lib() -> ctypes.CDLL:
     """The loaded C library (for callers that pass raw pointers)."""
     return _lib
@@ -216,6 +228,26 @@ def gemm(X, qw: QuantizedWeight, out_dtype=None, path: str = "auto", out=None, f
 
 
 DECODE_STATIC_SCRATCH_BYTES = 8 << 20
+
+
+def gemm_group(items, out_dtype=None, outs=None, flags=None, stream=None):
+    """One launch for several decode-step layers: items = [(X, qw), ...] with
+    bf16 X [M, K_i] (one M <= 16 for all) and packed layers of any b.
+    Returns the list of Y_i [M, N_i] (bf16 unless out_dtype says fp32)."""
+    import torch
+    out_dtype = out_dtype or torch.bfloat16
+    M = items[0][0].shape[0]
+    ys = outs if outs is not None else [
+        torch.empty((M, qw.N), dtype=out_dtype, device=X.device) for X, qw in items]
+    arr = (GemmLayer * len(items))()
+    for i, ((X, qw), y) in enumerate(zip(items, ys)):
+        assert X.dtype == torch.bfloat16 and X.is_cuda and X.is_contiguous() and X.shape == (M, qw.K)
+        arr[i] = GemmLayer(_ptr(X), qw.N, qw.K, qw.bits, _ptr(qw.packed), _ptr(qw.scales),
+                           _ptr(qw.zeros), _ptr(y))
+    dt = SLQ_DTYPE_F32 if ys[0].dtype == torch.float32 else SLQ_DTYPE_BF16
+    _check(_lib.slq_gemm_group(arr, len(items), M, dt, _ptr(flags), _stream_ptr(stream)),
+           "slq_gemm_group")
+    return ys
 
 
 def gemm_decode_static(X, qw: QuantizedWeight, out_dtype=None, out=None, flags=None, stream=None):

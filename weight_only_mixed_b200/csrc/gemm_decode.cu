@@ -727,21 +727,48 @@ constexpr int gemv_stage_bytes() {  // one warp's stage
   return GB * RT * 2 * 8 * 16 * B;
 }
 
+template <int B, int RT, int S>
+constexpr int gemv_depth() {  // stages per warp: about 6 KiB of ring per warp, 2..8
+  constexpr int d = 6 * 1024 / gemv_stage_bytes<B, RT, 2>();
+  return d < 2 ? 2 : d > 8 ? 8 : d;
+}
+
+template <int B, int RT, int S>
+constexpr bool gemv_fits() {  // the CTA's rings within 192 KiB
+  return S * gemv_depth<B, RT, S>() * gemv_stage_bytes<B, RT, 2>() <= 192 * 1024;
+}
+
+
+// One layer of a GEMV launch (all device pointers; gmax = the most groups a
+// warp takes, ceil(G / S)).
+struct GemvLayer {
+  const uint16_t* X;
+  const uint8_t* packed;
+  const uint16_t* scales;
+  const uint8_t* zeros;
+  void* Y;
+  int N, K, gmax, bits;
+};
+
+// Row tile `tile` of one layer, computed by the whole CTA.
 template <int B, int NT, int RT, int S, int GB, int D>
-__global__ void __launch_bounds__(32 * S)
-    gemm_gemv_kernel(const uint16_t* __restrict__ X, int M, int N, int K,
-                     const uint8_t* __restrict__ packed, const uint16_t* __restrict__ scales,
-                     const uint8_t* __restrict__ zeros, void* __restrict__ Y, int y_f32, int gmax) {
+__device__ __forceinline__ void gemv_tile(const GemvLayer& L, int M, int y_f32, int tile,
+                                          uint8_t* smem) {
+  const uint16_t* __restrict__ X = L.X;
+  const uint8_t* __restrict__ packed = L.packed;
+  const uint16_t* __restrict__ scales = L.scales;
+  const uint8_t* __restrict__ zeros = L.zeros;
+  void* __restrict__ Y = L.Y;
+  const int N = L.N, K = L.K, gmax = L.gmax;
   constexpr int kTile = 16 * RT;
   constexpr int kRowG = 16 * B;  // bytes of one row's group
   constexpr int kStage = gemv_stage_bytes<B, RT, GB>();
   constexpr bool kFold = B == 3 || B == 5 || B == 6 || B == 7;
-  extern __shared__ __align__(16) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = lane & 3, q = lane >> 2;
   const int G = K / kGroup;
   const int64_t row_bytes = static_cast<int64_t>(G) * kRowG;
-  const int tile0 = static_cast<int>(blockIdx.x) * kTile;
+  const int tile0 = tile * kTile;
   const int g0 = static_cast<int>(static_cast<int64_t>(G) * warp / S);
   const int g1 = static_cast<int>(static_cast<int64_t>(G) * (warp + 1) / S);
   const int ng = g1 - g0;
@@ -955,6 +982,42 @@ __global__ void __launch_bounds__(32 * S)
   }
 }
 
+template <int B, int NT, int RT, int S, int GB, int D>
+__global__ void __launch_bounds__(32 * S)
+    gemm_gemv_kernel(const __grid_constant__ GemvLayer L, int M, int y_f32) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  gemv_tile<B, NT, RT, S, GB, D>(L, M, y_f32, static_cast<int>(blockIdx.x), smem);
+}
+
+// Several layers (any mix of b, N, K) in one launch: the CTAs are the
+// layers' row tiles in order; each finds its layer and runs that layer's b.
+constexpr int kMaxGroup = 8;
+struct GemvGroup {
+  GemvLayer layer[kMaxGroup];
+  int tile_end[kMaxGroup];  // prefix sums of the layers' row tiles
+  int count;
+};
+
+template <int NT, int RT, int S>
+__global__ void __launch_bounds__(32 * S)
+    gemm_gemv_group_kernel(const __grid_constant__ GemvGroup grp, int M, int y_f32) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int cta = static_cast<int>(blockIdx.x);
+  int i = 0;
+  while (i + 1 < grp.count && cta >= grp.tile_end[i]) ++i;
+  const int tile = cta - (i ? grp.tile_end[i - 1] : 0);
+  const GemvLayer& L = grp.layer[i];
+  switch (L.bits) {
+    case 2: gemv_tile<2, NT, RT, S, 2, gemv_depth<2, RT, S>()>(L, M, y_f32, tile, smem); break;
+    case 3: gemv_tile<3, NT, RT, S, 2, gemv_depth<3, RT, S>()>(L, M, y_f32, tile, smem); break;
+    case 4: gemv_tile<4, NT, RT, S, 2, gemv_depth<4, RT, S>()>(L, M, y_f32, tile, smem); break;
+    case 5: gemv_tile<5, NT, RT, S, 2, gemv_depth<5, RT, S>()>(L, M, y_f32, tile, smem); break;
+    case 6: gemv_tile<6, NT, RT, S, 2, gemv_depth<6, RT, S>()>(L, M, y_f32, tile, smem); break;
+    case 7: gemv_tile<7, NT, RT, S, 2, gemv_depth<7, RT, S>()>(L, M, y_f32, tile, smem); break;
+    default: gemv_tile<8, NT, RT, S, 2, gemv_depth<8, RT, S>()>(L, M, y_f32, tile, smem); break;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
@@ -1085,17 +1148,6 @@ cudaError_t launch_gemm_decode(const uint16_t* X, int64_t M, int64_t N, int64_t 
 
 namespace {
 
-template <int B, int RT, int S>
-constexpr int gemv_depth() {  // stages per warp: about 6 KiB of ring per warp, 2..8
-  constexpr int d = 6 * 1024 / gemv_stage_bytes<B, RT, 2>();
-  return d < 2 ? 2 : d > 8 ? 8 : d;
-}
-
-template <int B, int RT, int S>
-constexpr bool gemv_fits() {  // the CTA's rings within 192 KiB
-  return S * gemv_depth<B, RT, S>() * gemv_stage_bytes<B, RT, 2>() <= 192 * 1024;
-}
-
 template <int B, int NT, int RT, int S>
 cudaError_t launch_gemv_cfg(const uint16_t* X, int M, int N, int K, const uint32_t* packed,
                             const uint16_t* scales, const uint8_t* zeros, void* Y, bool y_f32,
@@ -1127,8 +1179,8 @@ cudaError_t launch_gemv_cfg(const uint16_t* X, int M, int N, int K, const uint32
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, X, M, N, K, reinterpret_cast<const uint8_t*>(packed),
-                            scales, zeros, Y, y_f32 ? 1 : 0, gmax);
+  const GemvLayer L{X, reinterpret_cast<const uint8_t*>(packed), scales, zeros, Y, N, K, gmax, B};
+  return cudaLaunchKernelEx(&cfg, kern, L, M, y_f32 ? 1 : 0);
 }
 
 template <int B, int NT, int RT>
@@ -1188,6 +1240,130 @@ cudaError_t launch_gemm_gemv(const uint16_t* X, int64_t M, int64_t N, int64_t K,
     case 8: return launch_gemv_b<8>(X, m, n, k, packed, scales, zeros, Y, y_f32, stream);
     default: return cudaErrorInvalidValue;
   }
+}
+
+namespace {
+
+// Shared memory a layer of b bits needs in a CTA of the (NT, RT, S) shape,
+// and whether two ring stages per warp fit at all.
+template <int NT, int RT, int S>
+size_t gemv_group_smem(int b, int gmax, bool* fits) {
+  size_t stage = 0;
+  int d = 0;
+  bool f = false;
+  switch (b) {
+#define SLQ_GEMV_CASE(BB)                                    \
+  case BB:                                                   \
+    stage = gemv_stage_bytes<BB, RT, 2>();                   \
+    d = gemv_depth<BB, RT, S>();                             \
+    f = gemv_fits<BB, RT, S>();                              \
+    break;
+    SLQ_GEMV_CASE(2) SLQ_GEMV_CASE(3) SLQ_GEMV_CASE(4) SLQ_GEMV_CASE(5)
+    SLQ_GEMV_CASE(6) SLQ_GEMV_CASE(7) SLQ_GEMV_CASE(8)
+#undef SLQ_GEMV_CASE
+    default: break;
+  }
+  *fits = f;
+  const size_t rings = static_cast<size_t>(S) * d * stage;
+  const size_t szb = static_cast<size_t>(S) * 16 * RT * gmax * 4;
+  const size_t partb = static_cast<size_t>(S) * 16 * RT * (8 * NT + 1) * 4;
+  return (rings + szb) > partb ? rings + szb : partb;
+}
+
+template <int NT, int RT, int S>
+cudaError_t launch_group_cfg(const GemvLayer* layers, int count, int M, bool y_f32,
+                             cudaStream_t stream, bool* fits) {
+  GemvGroup grp = {};
+  grp.count = count;
+  size_t smem = 0;
+  int tiles = 0;
+  *fits = true;
+  for (int i = 0; i < count; ++i) {
+    grp.layer[i] = layers[i];
+    const int G = layers[i].K / kGroup;
+    grp.layer[i].gmax = (G + S - 1) / S;
+    bool f = false;
+    const size_t need = gemv_group_smem<NT, RT, S>(layers[i].bits, grp.layer[i].gmax, &f);
+    if (!f || need > 227 * 1024) {
+      *fits = false;
+      return cudaSuccess;
+    }
+    smem = need > smem ? need : smem;
+    tiles += (layers[i].N + 16 * RT - 1) / (16 * RT);
+    grp.tile_end[i] = tiles;
+  }
+  auto kern = gemm_gemv_group_kernel<NT, RT, S>;
+  static int attr_bytes = 0;  // per template instance: the largest size set so far
+  if (static_cast<int>(smem) > attr_bytes) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    attr_bytes = static_cast<int>(smem);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles), 1, 1);
+  cfg.blockDim = dim3(32 * S, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, grp, M, y_f32 ? 1 : 0);
+}
+
+// The same shape rules as a single layer, applied to the group's totals.
+template <int NT, int RT>
+cudaError_t launch_group_rt(const GemvLayer* layers, int count, int M, bool y_f32,
+                            cudaStream_t stream) {
+  int tiles = 0, gmin = 1 << 30;
+  for (int i = 0; i < count; ++i) {
+    tiles += (layers[i].N + 16 * RT - 1) / (16 * RT);
+    const int G = layers[i].K / kGroup;
+    gmin = G < gmin ? G : gmin;
+  }
+  bool fits = false;
+  cudaError_t e = cudaSuccess;
+  if ((NT == 2 ? tiles : tiles * RT) < 148 && gmin >= 32) {
+    e = launch_group_cfg<NT, RT, 16>(layers, count, M, y_f32, stream, &fits);
+    if (fits || e != cudaSuccess) return e;
+  }
+  if (tiles * RT < 600 && gmin >= 16) {
+    e = launch_group_cfg<NT, RT, 8>(layers, count, M, y_f32, stream, &fits);
+    if (fits || e != cudaSuccess) return e;
+  }
+  e = launch_group_cfg<NT, RT, 4>(layers, count, M, y_f32, stream, &fits);
+  if (e != cudaSuccess) return e;
+  return fits ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+int gemm_gemv_group_max() { return kMaxGroup; }
+
+cudaError_t launch_gemm_gemv_group(const GemvCall* calls, int count, int64_t M, bool y_f32,
+                                   cudaStream_t stream) {
+  if (count < 1 || count > kMaxGroup) return cudaErrorInvalidValue;
+  GemvLayer layers[kMaxGroup];
+  int64_t rows = 0;
+  int bmax = 0;
+  for (int i = 0; i < count; ++i) {
+    const GemvCall& c = calls[i];
+    layers[i] = GemvLayer{c.X, reinterpret_cast<const uint8_t*>(c.packed), c.scales, c.zeros, c.Y,
+                          static_cast<int>(c.N), static_cast<int>(c.K), 0, c.bits};
+    rows += c.N;
+    bmax = c.bits > bmax ? c.bits : bmax;
+  }
+  const int m = static_cast<int>(M);
+  // Two m16 tiles per warp on the rules of the single-layer launch.
+  if (m <= 8) {
+    if (bmax <= 6 && (rows + 31) / 32 >= 128)
+      return launch_group_rt<1, 2>(layers, count, m, y_f32, stream);
+    return launch_group_rt<1, 1>(layers, count, m, y_f32, stream);
+  }
+  if ((rows + 31) / 32 >= 128) return launch_group_rt<2, 2>(layers, count, m, y_f32, stream);
+  return launch_group_rt<2, 1>(layers, count, m, y_f32, stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -43,6 +43,23 @@ cudaError_t launch_gemm_gemv(const uint16_t* X, int64_t M, int64_t N, int64_t K,
                              const uint32_t* packed, const uint16_t* scales, const uint8_t* zeros,
                              void* Y, bool y_f32, cudaStream_t stream);
 
+// One layer of a grouped GEMV launch.
+struct GemvCall {
+  const uint16_t* X;
+  const uint32_t* packed;
+  const uint16_t* scales;
+  const uint8_t* zeros;
+  void* Y;
+  int64_t N, K;
+  int bits;
+};
+
+// Up to gemm_gemv_group_max() layers (any b, N, K; one M <= 16) in one
+// launch of the split-K GEMV kernel.
+int gemm_gemv_group_max();
+cudaError_t launch_gemm_gemv_group(const GemvCall* calls, int count, int64_t M, bool y_f32,
+                                   cudaStream_t stream);
+
 // Largest N the decode kernel accepts (the fixed tile-counter region).
 int64_t gemm_decode_max_n();
 

@@ -202,6 +202,44 @@ slq_status slq_gemm(const void* X_bf16, int64_t M, int64_t N, int64_t K, int bit
                      workspace, workspace_bytes, flags, stream);
 }
 
+int slq_gemm_group_max(void) { return slq::gemm_gemv_group_max(); }
+
+slq_status slq_gemm_group(const slq_gemm_layer* layers, int count, int64_t M, slq_dtype y_dtype,
+                          uint32_t* flags, void* stream) {
+  if (!layers || count < 1 || count > slq::gemm_gemv_group_max() || M < 0 || M > 16)
+    return SLQ_ERR_INVALID_ARGUMENT;
+  slq::GemvCall calls[16];
+  Range ins[16 * 4], outs[16];
+  int n = 0;
+  for (int i = 0; i < count; ++i) {
+    const slq_gemm_layer& L = layers[i];
+    const slq_status v = validate_gemm(L.X_bf16, M, L.N, L.K, L.bits, L.packed, L.scales_f16,
+                                       L.zeros, L.Y, y_dtype, SLQ_GEMM_GEMV, nullptr, 0, flags);
+    if (v != SLQ_OK) return v;
+    if (M == 0 || L.N == 0) continue;
+    const int64_t G = L.K / slq::kGroup;
+    ins[4 * n + 0] = range_of(L.X_bf16, M * L.K * 2);
+    ins[4 * n + 1] = range_of(L.packed, L.N * L.K * L.bits / 8);
+    ins[4 * n + 2] = range_of(L.scales_f16, L.N * G * 2);
+    ins[4 * n + 3] = range_of(L.zeros, L.N * G);
+    outs[n] = range_of(L.Y, M * L.N * (y_dtype == SLQ_DTYPE_F32 ? 4 : 2));
+    calls[n] = slq::GemvCall{static_cast<const uint16_t*>(L.X_bf16), L.packed,
+                             static_cast<const uint16_t*>(L.scales_f16), L.zeros, L.Y, L.N, L.K,
+                             L.bits};
+    ++n;
+  }
+  if (n == 0) return SLQ_OK;
+  if (!disjoint(outs, n, ins, 4 * n)) return SLQ_ERR_INVALID_ARGUMENT;
+  if (flags) {
+    const Range f = range_of(flags, 4);
+    if (!disjoint(&f, 1, ins, 4 * n) || !disjoint(&f, 1, outs, n)) return SLQ_ERR_INVALID_ARGUMENT;
+  }
+  const slq_status dev = check_device();
+  if (dev != SLQ_OK) return dev;
+  return from_cuda(slq::launch_gemm_gemv_group(calls, n, M, y_dtype == SLQ_DTYPE_F32,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
 slq_status slq_gemm_decode_static(const void* X_bf16, int64_t M, int64_t N, int64_t K, int bits,
                                   const uint32_t* packed, const void* scales_f16,
                                   const uint8_t* zeros, void* Y, slq_dtype y_dtype,
