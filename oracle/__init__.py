@@ -68,6 +68,8 @@ def _load():
         lib.oracle_gemm.restype = ctypes.c_int
         lib.oracle_ear_kl.argtypes = [P, P, P, I64, I64, ctypes.c_double, P, P]
         lib.oracle_ear_kl.restype = ctypes.c_int
+        lib.oracle_ear_kl_topk.argtypes = [P, P, P, I64, I64, I64, ctypes.c_double, P, P, P]
+        lib.oracle_ear_kl_topk.restype = ctypes.c_int
         _lib = lib
         return lib
 
@@ -169,3 +171,24 @@ def ear_kl(a_bf16, b_bf16, tau: float, rows=None):
     if rc != 0:
         raise ValueError("oracle_ear_kl rejected its arguments")
     return ear, kl
+
+
+def ear_kl_topk(a_bf16, b_bf16, k: int, tau: float, rows=None):
+    """Per-token top-K (EAR, KL, selected indices) in binary64."""
+    a = _u16(a_bf16)
+    b = _u16(b_bf16)
+    assert a.shape == b.shape and a.ndim == 2
+    T, V = a.shape
+    if rows is None:
+        n_rows, rows_arr = T, None
+    else:
+        rows_arr = np.ascontiguousarray(rows, dtype=np.int64)
+        n_rows = rows_arr.shape[0]
+    ear = np.empty(n_rows, dtype=np.float64)
+    kl = np.empty(n_rows, dtype=np.float64)
+    top = np.empty((n_rows, k), dtype=np.int64)
+    rc = _load().oracle_ear_kl_topk(_ptr(a), _ptr(b), None if rows_arr is None else _ptr(rows_arr),
+                                    n_rows, V, int(k), float(tau), _ptr(ear), _ptr(kl), _ptr(top))
+    if rc != 0:
+        raise ValueError("oracle_ear_kl_topk rejected its arguments")
+    return ear, kl, top

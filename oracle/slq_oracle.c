@@ -328,3 +328,80 @@ int oracle_ear_kl(const uint16_t *a_bf16, const uint16_t *b_bf16,
   free(y);
   return 0;
 }
+
+/*
+ * Top-K form of the same metrics, the one the pages' search and evaluation
+ * use: EAR = (1/N) sum_i sum_{k=1..K} min(p_i(k), q_i(k)) restricted to the
+ * top-K tokens (gist.science summary, Methodology section 2 "Fidelity
+ * Metrics", Definition; GitHub README "2. Build the sensitivity database":
+ * top-K = 10; eval/run_ear.py and eval/run_kl.py, "EAR and top-K KL").
+ *
+ * Readings (the pages leave them open):
+ *   - the top-K set T is the K tokens with the largest reference logits a
+ *     (the original model's distribution p), ties to the lower index;
+ *   - EAR sums min(p_v, q_v) over T with p and q the full-vocabulary
+ *     softmaxes (not renormalized), so it is at most the full EAR and equals
+ *     it when K = V;
+ *   - KL is KL(p_T || q_T) between p and q renormalized over T, a proper
+ *     divergence that equals the full KL when K = V.
+ * Selection is K passes of "largest remaining logit" over the row.
+ */
+int oracle_ear_kl_topk(const uint16_t *a_bf16, const uint16_t *b_bf16,
+                       const int64_t *rows, int64_t n_rows, int64_t V, int64_t K,
+                       double tau, double *ear, double *kl, int64_t *top) {
+  if (V < 1 || K < 1 || K > V || !(tau > 0.0) || isinf(tau)) return -1;
+  double *x = (double *)malloc((size_t)V * sizeof(double));
+  double *y = (double *)malloc((size_t)V * sizeof(double));
+  unsigned char *taken = (unsigned char *)calloc((size_t)V, 1);
+  int64_t *sel = (int64_t *)malloc((size_t)K * sizeof(int64_t));
+  if (!x || !y || !taken || !sel) {
+    free(x);
+    free(y);
+    free(taken);
+    free(sel);
+    return -2;
+  }
+  for (int64_t i = 0; i < n_rows; ++i) {
+    int64_t t = rows ? rows[i] : i;
+    for (int64_t v = 0; v < V; ++v) {
+      x[v] = (double)oracle_bf16_to_f32(a_bf16[t * V + v]) / tau;
+      y[v] = (double)oracle_bf16_to_f32(b_bf16[t * V + v]) / tau;
+      taken[v] = 0;
+    }
+    /* T: K passes, each taking the largest remaining a (lowest index on ties). */
+    for (int64_t k = 0; k < K; ++k) {
+      int64_t best = -1;
+      for (int64_t v = 0; v < V; ++v) {
+        if (taken[v]) continue;
+        if (best < 0 || x[v] > x[best]) best = v;
+      }
+      taken[best] = 1;
+      sel[k] = best;
+      if (top) top[i * K + k] = best;
+    }
+    double la = logsumexp(x, V);
+    double lb = logsumexp(y, V);
+    double e = 0.0, pt = 0.0, qt = 0.0;
+    for (int64_t k = 0; k < K; ++k) {
+      double p = exp(x[sel[k]] - la);
+      double q = exp(y[sel[k]] - lb);
+      e += (p < q) ? p : q;
+      pt += p;
+      qt += q;
+    }
+    /* KL(p_T || q_T) with p_T = p / pt, q_T = q / qt, from the log-softmax. */
+    double d = 0.0;
+    for (int64_t k = 0; k < K; ++k) {
+      double log_pt = (x[sel[k]] - la) - log(pt);
+      double log_qt = (y[sel[k]] - lb) - log(qt);
+      d += exp(log_pt) * (log_pt - log_qt);
+    }
+    ear[i] = e;
+    kl[i] = d;
+  }
+  free(x);
+  free(y);
+  free(taken);
+  free(sel);
+  return 0;
+}

@@ -77,6 +77,14 @@ int oracle_ear_kl(const uint16_t *a_bf16, const uint16_t *b_bf16,
                   const int64_t *rows, int64_t n_rows, int64_t V, double tau,
                   double *ear, double *kl);
 
+/* Top-K EAR and KL (readings in slq_oracle.c): T = the K largest a (ties to
+ * the lower index); ear = sum over T of min(p, q) with full softmaxes; kl =
+ * KL between p and q renormalized over T.  top (nullable): [n_rows, K] the
+ * selected token indices, largest first. */
+int oracle_ear_kl_topk(const uint16_t *a_bf16, const uint16_t *b_bf16,
+                       const int64_t *rows, int64_t n_rows, int64_t V, int64_t K,
+                       double tau, double *ear, double *kl, int64_t *top);
+
 #ifdef __cplusplus
 }
 #endif

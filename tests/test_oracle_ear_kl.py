@@ -105,3 +105,60 @@ def test_sampled_rows_and_single_token_vocab():
     two = synth.to_bf16_bits(np.array([[1.0], [5.0]]))
     ear, kl = oracle.ear_kl(one, two, 1.0)
     assert np.all(ear == 1.0) and np.all(kl == 0.0)
+
+
+# ---------------------------------------------------------------------------
+# Top-K form (T = the K largest reference logits, ties to the lower index;
+# EAR over T with full softmaxes; KL between p and q renormalized over T).
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("tau", [1.0, 0.7])
+def test_topk_with_k_equal_v_is_the_full_metric(tau):
+    a, b = synth.logits(4, 777, seed=21)
+    e, k, top = oracle.ear_kl_topk(a, b, 777, tau)
+    E, K = oracle.ear_kl(a, b, tau)
+    assert np.allclose(e, E, rtol=0, atol=1e-12) and np.allclose(k, K, rtol=0, atol=1e-12)
+    assert all(sorted(r) == list(range(777)) for r in top)
+
+
+@pytest.mark.parametrize("K", [1, 3, 10, 32])
+@pytest.mark.parametrize("tau", [1.0, 0.7])
+def test_topk_matches_scipy_on_the_selected_set(K, tau):
+    a, b = synth.logits(5, 1500, seed=31 + K)
+    e, k, top = oracle.ear_kl_topk(a, b, K, tau)
+    for i in range(a.shape[0]):
+        x, y = _vals(a[i]), _vals(b[i])
+        order = np.argsort(-x, kind="stable")[:K]  # stable: ties keep the lower index first
+        assert np.array_equal(top[i], order)
+        p, q = softmax(x / tau), softmax(y / tau)
+        assert abs(e[i] - np.minimum(p[order], q[order]).sum()) <= 1e-12
+        pt, qt = p[order] / p[order].sum(), q[order] / q[order].sum()
+        assert abs(k[i] - entropy(pt, qt)) <= 1e-12
+
+
+def test_topk_ties_take_the_lower_index():
+    x = np.array([[1.0, 3.0, 3.0, 2.0, 3.0, -1.0, 2.0, 2.0]])
+    bits = synth.to_bf16_bits(x)
+    _, _, top = oracle.ear_kl_topk(bits, bits, 5, 1.0)
+    assert top[0].tolist() == [1, 2, 4, 3, 6]
+
+
+def test_topk_invariants():
+    a, b = synth.logits(6, 900, seed=41)
+    for K in (1, 2, 10):
+        e_aa, k_aa, top = oracle.ear_kl_topk(a, a, K, 1.0)
+        p_mass = np.array([softmax(_vals(a[i]))[top[i]].sum() for i in range(a.shape[0])])
+        assert np.allclose(e_aa, p_mass, atol=1e-12)  # EAR(p, p) over T = p(T)
+        assert np.abs(k_aa).max() <= 1e-12  # KL(p, p) = 0
+    # K = 1: min(p_top, q_top); the renormalized one-point distributions agree.
+    e1, k1, top1 = oracle.ear_kl_topk(a, b, 1, 1.0)
+    for i in range(a.shape[0]):
+        v = top1[i, 0]
+        assert abs(e1[i] - min(softmax(_vals(a[i]))[v], softmax(_vals(b[i]))[v])) <= 1e-12
+    assert np.abs(k1).max() <= 1e-15
+    # EAR over T grows with K and stays below the full EAR.
+    E, _ = oracle.ear_kl(a, b, 1.0)
+    prev = np.zeros(a.shape[0])
+    for K in (1, 2, 5, 10, 50, 900):
+        e, _, _ = oracle.ear_kl_topk(a, b, K, 1.0)
+        assert np.all(e >= prev - 1e-15) and np.all(e <= E + 1e-12)
+        prev = e
