@@ -28,6 +28,7 @@ ncu captures use.  SPEC is one of
   decode:N:K:b:M            one dequant-GEMM on the stream-K decode kernel (M <= 16)
   tiled:N:K:b:M             one dequant-GEMM on the tiled tcgen05 kernel
   ear:T:V:tau               one EAR/KL reduction
+  eartopk:T:V:tau:K         one top-K EAR/KL reduction
   quantize:N:K:b            one quantize+pack
 
 --impl reference times the CPU oracle (the plain reference implementation
@@ -525,6 +526,18 @@ def other_rows(args, slq, synth, torch, dev, stream, hbm_peak, tc_peak, rank):
                                     "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / hbm_peak, 3),
                                     "us": round(ms * 1e3, 1), "ear_mean": round(em.item(), 6),
                                     "kl_mean": round(km.item(), 7)}
+    # Top-K form (K = 10, the pages' evaluation), one pass over the logits.
+    for tau in (1.0,):
+        def f():
+            rc = L.slq_ear_kl_topk(a.data_ptr(), bq.data_ptr(), T, V, 10, tau, ear.data_ptr(),
+                                   kl.data_ptr(), em.data_ptr(), km.data_ptr(), None, stream.cuda_stream)
+            assert rc == 0
+        ms = time_ms(torch, stream, f, 5, warm=1)
+        nbytes = 2 * T * V * 2
+        rows[f"ear_kl_top10_tau{tau}"] = {"GBps": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                                          "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / hbm_peak, 3),
+                                          "us": round(ms * 1e3, 1), "ear_mean": round(em.item(), 6),
+                                          "kl_mean": round(km.item(), 7)}
     del a, bq
     return rows
 
@@ -656,6 +669,13 @@ def run_case(args):
         def fn():
             slq.ear_kl(a, bq, float(tau), stream=stream)
         per_call = 2  # the reduction and the token means
+    elif kind == "eartopk":
+        T, V, tau, k = vals
+        a, bq = synth.logits_torch(T, V, device=dev)
+
+        def fn():
+            slq.ear_kl(a, bq, float(tau), top_k=int(k), stream=stream)
+        per_call = 2
     elif kind == "quantize":
         N, K, b = vals
         W = synth.weights_torch(N, K, device=dev)

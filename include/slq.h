@@ -283,6 +283,28 @@ slq_status slq_ear_kl(const void *logits_p_bf16, const void *logits_q_bf16,
                       float *kl_tok, double *ear_mean, double *kl_mean,
                       uint32_t *flags, void *stream);
 
+/*
+ * slq_ear_kl_topk -- the top-K form of slq_ear_kl, the one the pages' search
+ * and evaluation use: EAR = (1/N) sum_i sum_{k=1..K} min(p_i(k), q_i(k))
+ * restricted to the top-K tokens (gist.science summary, Methodology section 2
+ * "Fidelity Metrics", Definition; GitHub README "2. Build the sensitivity
+ * database": top-K = 10).  Readings where the pages are open: the top-K set
+ * T_t is the K largest reference logits of token t (ties to the lower
+ * index); EAR sums min(p, q) over T_t with p, q the full-vocabulary
+ * softmaxes; KL is KL(p_T || q_T) with p and q renormalized over T_t.  With
+ * K = V both equal slq_ear_kl.
+ *
+ * top_k        1 .. min(V, slq_ear_kl_topk_max()) (16); other arguments,
+ *              layouts and errors as for slq_ear_kl.
+ */
+slq_status slq_ear_kl_topk(const void *logits_p_bf16, const void *logits_q_bf16,
+                           int64_t T, int64_t V, int top_k, float temperature,
+                           float *ear_tok, float *kl_tok, double *ear_mean,
+                           double *kl_mean, uint32_t *flags, void *stream);
+
+/* Largest top_k slq_ear_kl_topk takes (16). */
+int slq_ear_kl_topk_max(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -173,3 +173,17 @@ def test_gemm_group_validation():
                                            FAKE + (10 << 24), FAKE + (11 << 24), FAKE + (4 << 24))]),
     ]
     assert all(r == slq.SLQ_ERR_INVALID_ARGUMENT for r in bad), bad
+
+
+def test_ear_kl_topk_validation():
+    assert L.slq_ear_kl_topk_max() == 16
+
+    def call(T=4, V=1000, k=10, tau=1.0, a=FAKE, b=FAKE + (1 << 24), ear=FAKE + (2 << 24),
+             kl=FAKE + (3 << 24)):
+        return L.slq_ear_kl_topk(a, b, T, V, k, tau, ear, kl, None, None, None, None)
+
+    for bad in [dict(k=0), dict(k=17), dict(V=5, k=6), dict(tau=0.0), dict(a=None), dict(ear=FAKE + 8),
+                dict(a=FAKE + 2)]:
+        assert call(**bad) == slq.SLQ_ERR_INVALID_ARGUMENT, bad
+    assert call(T=0) == slq.SLQ_OK
+    assert call() in (slq.SLQ_OK, slq.SLQ_ERR_UNSUPPORTED_DEVICE)

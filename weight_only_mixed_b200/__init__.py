@@ -90,6 +90,10 @@ _lib.slq_gemm_group.argtypes = [ctypes.POINTER(GemmLayer), _I, _I64, _I, _P, _P]
 _lib.slq_gemm_group.restype = _I
 _lib.slq_gemm_group_max.argtypes = []
 _lib.slq_gemm_group_max.restype = _I
+_lib.slq_ear_kl_topk.argtypes = [_P, _P, _I64, _I64, _I, ctypes.c_float, _P, _P, _P, _P, _P, _P]
+_lib.slq_ear_kl_topk.restype = _I
+_lib.slq_ear_kl_topk_max.argtypes = []
+_lib.slq_ear_kl_topk_max.restype = _I
 
 
 def lib() -> ctypes.CDLL:
@@ -266,8 +270,10 @@ def gemm_decode_static(X, qw: QuantizedWeight, out_dtype=None, out=None, flags=N
     return y
 
 
-def ear_kl(a, b, temperature: float = 1.0, means: bool = True, flags=None, stream=None):
-    """Per-token EAR and KL(p || q) of two [T, V] bf16 logit tensors.
+def ear_kl(a, b, temperature: float = 1.0, means: bool = True, flags=None, stream=None,
+           top_k: int | None = None):
+    """Per-token EAR and KL(p || q) of two [T, V] bf16 logit tensors; with
+    top_k, the top-K form (slq_ear_kl_topk).
 
     Returns (ear_tok, kl_tok, ear_mean, kl_mean); the means are 0-d float64
     tensors on the device (None when means=False)."""
@@ -279,6 +285,11 @@ def ear_kl(a, b, temperature: float = 1.0, means: bool = True, flags=None, strea
     kl = torch.empty(T, dtype=torch.float32, device=a.device)
     em = torch.empty((), dtype=torch.float64, device=a.device) if means else None
     km = torch.empty((), dtype=torch.float64, device=a.device) if means else None
+    if top_k is not None:
+        _check(_lib.slq_ear_kl_topk(_ptr(a), _ptr(b), T, V, int(top_k), float(temperature), _ptr(ear),
+                                    _ptr(kl), _ptr(em), _ptr(km), _ptr(flags), _stream_ptr(stream)),
+               "slq_ear_kl_topk")
+        return ear, kl, em, km
     _check(_lib.slq_ear_kl(_ptr(a), _ptr(b), T, V, float(temperature), _ptr(ear), _ptr(kl),
                            _ptr(em), _ptr(km), _ptr(flags), _stream_ptr(stream)), "slq_ear_kl")
     return ear, kl, em, km

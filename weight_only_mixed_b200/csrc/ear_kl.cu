@@ -17,6 +17,8 @@
 // is one rounding away from exact.
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -569,6 +571,217 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Top-K form (the pages' evaluation: EAR and KL restricted to the top-K
+// tokens).  T = the K largest reference logits a, ties to the lower index;
+// EAR = sum over T of min(p, q) with the full-vocabulary softmaxes; KL =
+// KL(p_T || q_T) with p and q renormalized over T.
+//
+// One CTA per row, one pass over the row: every thread keeps the online
+// statistics of its logits (as above) and a sorted register list of its KM
+// best (a, index) pairs (KM = the power of two >= K, so the list covers the
+// top K), only checking a unit's 8 logits when the unit's maximum (packed
+// bf16 max) reaches the list's last entry.  Warps then merge their
+// lanes' lists by K rounds of a shuffle arg-max, warp 0 merges the warps'
+// lists the same way, and K lanes form the terms from the row statistics.
+// ---------------------------------------------------------------------------
+constexpr int kTopMax = 16;
+constexpr int kTopThreads = 512;
+
+// (v, i) ranks before (w, j): larger logit first, lower index on ties.
+__device__ __forceinline__ bool top_before(float v, int i, float w, int j) {
+  return v > w || (v == w && i < j);
+}
+
+template <int KM>
+struct TopList {
+  float v[KM];
+  int i[KM];
+};
+
+template <int KM>
+__device__ __forceinline__ void top_init(TopList<KM>& t) {
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    t.v[j] = -INFINITY;
+    t.i[j] = 0x7fffffff;
+  }
+}
+
+// Insert (v, i) into the sorted list; no-op if it ranks after the last entry.
+template <int KM>
+__device__ __forceinline__ void top_push(TopList<KM>& t, float v, int i) {
+  if (!top_before(v, i, t.v[KM - 1], t.i[KM - 1])) return;
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    if (top_before(v, i, t.v[j], t.i[j])) {
+      const float tv = t.v[j];
+      const int ti = t.i[j];
+      t.v[j] = v;
+      t.i[j] = i;
+      v = tv;
+      i = ti;
+    }
+  }
+}
+
+// K rounds of a warp arg-max over the lanes' sorted lists (each lane's head
+// advances when it wins); lane r < K ends with the r-th best of the warp.
+template <int KM>
+__device__ __forceinline__ void top_warp_merge(const TopList<KM>& t, int K, float& out_v,
+                                               int& out_i) {
+  const int lane = threadIdx.x & 31;
+  int h = 0;
+  out_v = -INFINITY;
+  out_i = 0x7fffffff;
+  for (int r = 0; r < K; ++r) {
+    float hv = -INFINITY;
+    int hi = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < KM; ++j)
+      if (j == h) {
+        hv = t.v[j];
+        hi = t.i[j];
+      }
+
+    float bv = hv;
+    int bi = hi, bl = lane;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(kFull, bv, off);
+      const int oi = __shfl_xor_sync(kFull, bi, off);
+      const int ol = __shfl_xor_sync(kFull, bl, off);
+      if (top_before(ov, oi, bv, bi) || (ov == bv && oi == bi && ol < bl)) {
+        bv = ov;
+        bi = oi;
+        bl = ol;
+      }
+    }
+    if (lane == bl) ++h;
+    if (lane == r) {
+      out_v = bv;
+      out_i = bi;
+    }
+  }
+}
+
+template <bool kVec, int KM>
+__global__ void __launch_bounds__(kTopThreads)
+    ear_kl_topk_kernel(const uint16_t* __restrict__ A, const uint16_t* __restrict__ Bq, int64_t T,
+                       int64_t V, int K, float c, float* __restrict__ ear_tok,
+                       float* __restrict__ kl_tok) {
+  constexpr int kWarps = kTopThreads / 32;
+  __shared__ Part parts[kWarps];
+  __shared__ float wv[kWarps][KM];
+  __shared__ int wi[kWarps][KM];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr float kLn2 = 0.693147180559945309f;
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    const uint16_t* a_row = A + t * V;
+    const uint16_t* b_row = Bq + t * V;
+    TopList<KM> top;
+    top_init(top);
+    RowStat st;
+    if constexpr (kVec) {
+      const int64_t nv = V / 8;
+      VecStat vs = vec_stat_init(c);
+      auto visit = [&](const uint4& va, int64_t unit) {
+        const uint4 one[1] = {va};
+        if (!(units_max<1>(one) >= top.v[KM - 1])) return;
+        const uint32_t w[4] = {va.x, va.y, va.z, va.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float x = (e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]);
+          top_push(top, x, static_cast<int>(8 * unit + e));
+        }
+      };
+      int64_t i = threadIdx.x;
+      for (; i + 3 * kTopThreads < nv; i += 4 * kTopThreads) {
+        uint4 va[4], vb[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          va[u] = ld_stream_v4(a_row + 8 * (i + u * kTopThreads));
+          vb[u] = ld_stream_v4(b_row + 8 * (i + u * kTopThreads));
+        }
+        push_units<4>(vs, va, vb, c);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) visit(va[u], i + u * kTopThreads);
+      }
+      for (; i < nv; i += kTopThreads) {
+        const uint4 va[1] = {ld_stream_v4(a_row + 8 * i)};
+        const uint4 vb[1] = {ld_stream_v4(b_row + 8 * i)};
+        push_units<1>(vs, va, vb, c);
+        visit(va[0], i);
+      }
+      st = vec_stat_final(vs, c);
+    } else {
+      st = RowStat{{-INFINITY, 0.0f}, {-INFINITY, 0.0f}, 0.0f};
+      for (int64_t v = threadIdx.x; v < V; v += kTopThreads) {
+        const float a = __uint_as_float(static_cast<uint32_t>(a_row[v]) << 16);
+        const float b = __uint_as_float(static_cast<uint32_t>(b_row[v]) << 16);
+        push(st, a, b, c);
+        top_push(top, a, static_cast<int>(v));
+      }
+    }
+    // Row statistics and the warps' top-K lists.
+    Part mine{st, 0.0f};
+    mine = warp_reduce(mine, c);
+    float mv;
+    int mi;
+    top_warp_merge(top, K, mv, mi);
+    if (lane == 0) parts[warp] = mine;
+    if (lane < K) {
+      wv[warp][lane] = mv;
+      wi[warp][lane] = mi;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      Part tot = (lane < kWarps) ? parts[lane]
+                                 : Part{{{-INFINITY, 0.0f}, {-INFINITY, 0.0f}, 0.0f}, 0.0f};
+      tot = warp_reduce(tot, c);
+      TopList<KM> wl;
+      top_init(wl);
+      if (lane < kWarps) {
+#pragma unroll
+        for (int j = 0; j < KM; ++j)
+          if (j < K) {
+            wl.v[j] = wv[lane][j];
+            wl.i[j] = wi[lane][j];
+          }
+      }
+      float bv;
+      int bi;
+      top_warp_merge(wl, K, bv, bi);
+      // Lane k < K holds the k-th token of T: its terms in base 2.
+      const float la = lg2(tot.st.a.s), lb = lg2(tot.st.b.s);
+      float xa = -INFINITY, xb = -INFINITY;
+      if (lane < K && bi < V) {  // bi < V always holds for finite logits
+        const float a = __uint_as_float(static_cast<uint32_t>(a_row[bi]) << 16);
+        const float b = __uint_as_float(static_cast<uint32_t>(b_row[bi]) << 16);
+        xa = (a - tot.st.a.m) * c - la;  // log2 p
+        xb = (b - tot.st.b.m) * c - lb;  // log2 q
+      }
+      const float p = lane < K ? ex2(xa) : 0.0f, q = lane < K ? ex2(xb) : 0.0f;
+      float e = fminf(p, q), pt = p, qt = q;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        e += __shfl_xor_sync(kFull, e, off);
+        pt += __shfl_xor_sync(kFull, pt, off);
+        qt += __shfl_xor_sync(kFull, qt, off);
+      }
+      const float lpt = xa - lg2(pt), lqt = xb - lg2(qt);  // log2 of the renormalized p, q
+      float d = lane < K ? ex2(lpt) * (lpt - lqt) : 0.0f;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(kFull, d, off);
+      if (lane == 0) {
+        ear_tok[t] = e;
+        kl_tok[t] = d * kLn2;
+      }
+    }
+    __syncthreads();
+  }
+}
+
 // Means over tokens in binary64, one block, fixed summation order.
 __global__ void __launch_bounds__(1024)
     token_mean_kernel(const float* __restrict__ ear_tok, const float* __restrict__ kl_tok,
@@ -596,6 +809,41 @@ __global__ void __launch_bounds__(1024)
 }
 
 }  // namespace
+
+cudaError_t launch_ear_kl_topk(const uint16_t* a, const uint16_t* b, int64_t T, int64_t V, int K,
+                               float temperature, float* ear_tok, float* kl_tok, double* ear_mean,
+                               double* kl_mean, cudaStream_t stream) {
+  if (K < 1 || K > kTopMax || K > V) return cudaErrorInvalidValue;
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const float c = 1.4426950408889634f / temperature;
+  const int64_t cap = 2 * static_cast<int64_t>(sms);
+  const unsigned blocks = static_cast<unsigned>(T < cap ? T : cap);
+  const bool aligned = ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b)) & 15u) == 0;
+  const bool vec = V % 8 == 0 && aligned;
+  auto run = [&](auto km) {
+    constexpr int KM = decltype(km)::value;
+    if (vec)
+      ear_kl_topk_kernel<true, KM><<<blocks, kTopThreads, 0, stream>>>(a, b, T, V, K, c, ear_tok, kl_tok);
+    else
+      ear_kl_topk_kernel<false, KM><<<blocks, kTopThreads, 0, stream>>>(a, b, T, V, K, c, ear_tok, kl_tok);
+  };
+  if (K <= 1) run(std::integral_constant<int, 1>{});
+  else if (K <= 2) run(std::integral_constant<int, 2>{});
+  else if (K <= 4) run(std::integral_constant<int, 4>{});
+  else if (K <= 8) run(std::integral_constant<int, 8>{});
+  else run(std::integral_constant<int, 16>{});
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  if (ear_mean || kl_mean) {
+    token_mean_kernel<<<1, 1024, 0, stream>>>(ear_tok, kl_tok, T, ear_mean, kl_mean);
+    err = cudaGetLastError();
+  }
+  return err;
+}
+
+int ear_kl_topk_max() { return kTopMax; }
 
 cudaError_t launch_ear_kl(const uint16_t* a, const uint16_t* b, int64_t T, int64_t V,
                           float temperature, float* ear_tok, float* kl_tok, double* ear_mean,

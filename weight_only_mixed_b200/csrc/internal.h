@@ -85,4 +85,10 @@ cudaError_t launch_ear_kl(const uint16_t* a, const uint16_t* b, int64_t T, int64
                           double* ear_mean, double* kl_mean, uint32_t* flags,
                           cudaStream_t stream);
 
+// Top-K EAR / KL(p_T || q_T) over the K largest reference logits, K <= ear_kl_topk_max().
+int ear_kl_topk_max();
+cudaError_t launch_ear_kl_topk(const uint16_t* a, const uint16_t* b, int64_t T, int64_t V, int K,
+                               float temperature, float* ear_tok, float* kl_tok, double* ear_mean,
+                               double* kl_mean, cudaStream_t stream);
+
 }  // namespace slq

@@ -260,6 +260,46 @@ slq_status slq_gemm_decode_static(const void* X_bf16, int64_t M, int64_t N, int6
       static_cast<cudaStream_t>(stream)));
 }
 
+namespace {
+// Shared argument checks of slq_ear_kl and slq_ear_kl_topk.
+slq_status validate_ear(const void* logits_p_bf16, const void* logits_q_bf16, int64_t T, int64_t V,
+                        float temperature, float* ear_tok, float* kl_tok, double* ear_mean,
+                        double* kl_mean, uint32_t* flags) {
+  if (T < 0 || T > kMaxDim || V < 1 || V > kMaxDim || !product_ok(T, V))
+    return SLQ_ERR_INVALID_ARGUMENT;
+  if (!std::isfinite(temperature) || !(temperature > 0.0f)) return SLQ_ERR_INVALID_ARGUMENT;
+  if (T == 0) return SLQ_OK;
+  if (!logits_p_bf16 || !logits_q_bf16 || !ear_tok || !kl_tok) return SLQ_ERR_INVALID_ARGUMENT;
+  if (!aligned(logits_p_bf16, 16) || !aligned(logits_q_bf16, 16) || !aligned(ear_tok, 4) ||
+      !aligned(kl_tok, 4) || (ear_mean && !aligned(ear_mean, 8)) ||
+      (kl_mean && !aligned(kl_mean, 8)) || (flags && !aligned(flags, 4)))
+    return SLQ_ERR_INVALID_ARGUMENT;
+  const Range ins[2] = {range_of(logits_p_bf16, T * V * 2), range_of(logits_q_bf16, T * V * 2)};
+  const Range outs[5] = {range_of(ear_tok, T * 4), range_of(kl_tok, T * 4),
+                         range_of(ear_mean, ear_mean ? 8 : 0), range_of(kl_mean, kl_mean ? 8 : 0),
+                         range_of(flags, flags ? 4 : 0)};
+  if (!disjoint(outs, 5, ins, 2)) return SLQ_ERR_INVALID_ARGUMENT;
+  return SLQ_OK;
+}
+}  // namespace
+
+int slq_ear_kl_topk_max(void) { return slq::ear_kl_topk_max(); }
+
+slq_status slq_ear_kl_topk(const void* logits_p_bf16, const void* logits_q_bf16, int64_t T,
+                           int64_t V, int top_k, float temperature, float* ear_tok, float* kl_tok,
+                           double* ear_mean, double* kl_mean, uint32_t* flags, void* stream) {
+  if (top_k < 1 || top_k > slq::ear_kl_topk_max() || top_k > V || V > 0x7fffffff)
+    return SLQ_ERR_INVALID_ARGUMENT;
+  const slq_status v = validate_ear(logits_p_bf16, logits_q_bf16, T, V, temperature, ear_tok,
+                                    kl_tok, ear_mean, kl_mean, flags);
+  if (v != SLQ_OK || T == 0) return v;
+  const slq_status dev = check_device();
+  if (dev != SLQ_OK) return dev;
+  return from_cuda(slq::launch_ear_kl_topk(
+      static_cast<const uint16_t*>(logits_p_bf16), static_cast<const uint16_t*>(logits_q_bf16), T,
+      V, top_k, temperature, ear_tok, kl_tok, ear_mean, kl_mean, static_cast<cudaStream_t>(stream)));
+}
+
 slq_status slq_ear_kl(const void* logits_p_bf16, const void* logits_q_bf16, int64_t T, int64_t V,
                       float temperature, float* ear_tok, float* kl_tok, double* ear_mean,
                       double* kl_mean, uint32_t* flags, void* stream) {
