@@ -578,12 +578,13 @@ __global__ void __launch_bounds__(kThreads)
 // KL(p_T || q_T) with p and q renormalized over T.
 //
 // One CTA per row, one pass over the row: every thread keeps the online
-// statistics of its logits (as above) and a sorted register list of its KM
-// best (a, index) pairs (KM = the power of two >= K, so the list covers the
-// top K), only checking a unit's 8 logits when the unit's maximum (packed
-// bf16 max) reaches the list's last entry.  Warps then merge their
-// lanes' lists by K rounds of a shuffle arg-max, warp 0 merges the warps'
-// lists the same way, and K lanes form the terms from the row statistics.
+// statistics of its logits (as above).  Each warp keeps its top-K list in
+// registers across its lanes and a warp-wide threshold (the list's K-th
+// entry): a unit's 8 logits are offered only when the unit's maximum (packed
+// bf16 max) reaches the threshold, and offered logits that still reach it
+// are inserted with one shuffle.  After the row, warp 0 merges the warps'
+// lists by K rounds of a shuffle arg-max (KM = the power of two >= K bounds
+// the register lists), and K lanes form the terms.
 // ---------------------------------------------------------------------------
 constexpr int kTopMax = 16;
 constexpr int kTopThreads = 512;
@@ -665,6 +666,36 @@ __device__ __forceinline__ void top_warp_merge(const TopList<KM>& t, int K, floa
   }
 }
 
+// The warp's top-K list lives in registers across the lanes: lane r < K
+// holds the r-th best (a, index) seen by the warp so far, lanes >= K hold
+// placeholders.  Inserting a warp-uniform (v, i) shifts the entries that rank
+// after it down by one lane.
+__device__ __forceinline__ void warp_list_insert(float& lv, int& li, float v, int i) {
+  const int lane = threadIdx.x & 31;
+  const bool after = top_before(v, i, lv, li);  // this lane's entry now ranks after (v, i)
+  const float pv = __shfl_up_sync(kFull, lv, 1);
+  const int pi = __shfl_up_sync(kFull, li, 1);
+  const bool pafter = __shfl_up_sync(kFull, after ? 1 : 0, 1) != 0 && lane > 0;
+  if (after) {
+    lv = pafter ? pv : v;
+    li = pafter ? pi : i;
+  }
+}
+
+// The K-th largest of one value per lane (a bitonic sort over the warp).
+__device__ __forceinline__ float warp_kth_largest(float m, int K) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const float o = __shfl_xor_sync(kFull, m, j);
+      const bool up = (lane & k) == 0, lower = (lane & j) == 0;
+      m = (lower == up) ? fmaxf(m, o) : fminf(m, o);
+    }
+  return __shfl_sync(kFull, m, K - 1);
+}
+
 template <bool kVec, int KM>
 __global__ void __launch_bounds__(kTopThreads)
     ear_kl_topk_kernel(const uint16_t* __restrict__ A, const uint16_t* __restrict__ Bq, int64_t T,
@@ -679,24 +710,67 @@ __global__ void __launch_bounds__(kTopThreads)
   for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
     const uint16_t* a_row = A + t * V;
     const uint16_t* b_row = Bq + t * V;
-    TopList<KM> top;
-    top_init(top);
+    // thr: the warp's K-th best so far (or a lower bound of it); a logit
+    // below it cannot enter the row's top K.
+    float lv = -INFINITY, thr = -INFINITY;
+    int li = 0x7fffffff;
+    // Lanes whose `hit` is set offer their `cnt` logits (values from `get`)
+    // one at a time, in lane order; many hits first raise the threshold to
+    // the K-th largest of the lanes' maxima (at least K logits reach it).
+    // `sel(thr)` gives a lane's bitmask of its logits that reach thr.
+    auto offer = [&](bool hit, float mx, auto&& get, auto&& sel) {
+      unsigned mask = __ballot_sync(kFull, hit);
+      if (!mask) return;
+      if (__popc(mask) >= K && __popc(mask) > 4) {
+        thr = fmaxf(thr, warp_kth_largest(hit ? mx : -INFINITY, K));
+        mask = __ballot_sync(kFull, hit && mx >= thr);
+      }
+      const unsigned mine = (mask >> lane) & 1u ? sel(thr) : 0u;
+      while (mask) {
+        const int src = __ffs(mask) - 1;
+        mask &= mask - 1;
+        unsigned bits = __shfl_sync(kFull, mine, src);
+        while (bits) {
+          const int e = __ffs(bits) - 1;
+          bits &= bits - 1;
+          float x;
+          int ix;
+          get(src, e, x, ix);
+          if (x >= thr) {
+            warp_list_insert(lv, li, x, ix);
+            thr = fmaxf(thr, __shfl_sync(kFull, lv, K - 1));
+          }
+        }
+      }
+    };
     RowStat st;
     if constexpr (kVec) {
       const int64_t nv = V / 8;
       VecStat vs = vec_stat_init(c);
-      auto visit = [&](const uint4& va, int64_t unit) {
+      auto visit = [&](const uint4& va, int64_t unit, bool valid) {
         const uint4 one[1] = {va};
-        if (!(units_max<1>(one) >= top.v[KM - 1])) return;
-        const uint32_t w[4] = {va.x, va.y, va.z, va.w};
+        const float mx = valid ? units_max<1>(one) : -INFINITY;
+        offer(valid && mx >= thr, mx,
+              [&](int src, int e, float& x, int& ix) {
+                const uint32_t wsel = (e >> 1) == 0 ? va.x : (e >> 1) == 1 ? va.y : (e >> 1) == 2 ? va.z : va.w;
+                const uint32_t w = __shfl_sync(kFull, wsel, src);
+                x = (e & 1) ? bf16_hi(w) : bf16_lo(w);
+                ix = 8 * static_cast<int>(__shfl_sync(kFull, static_cast<int>(unit), src)) + e;
+              },
+              [&](float th) {
+                const uint32_t w[4] = {va.x, va.y, va.z, va.w};
+                unsigned bits = 0;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float x = (e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]);
-          top_push(top, x, static_cast<int>(8 * unit + e));
-        }
+                for (int e = 0; e < 8; ++e)
+                  if (((e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1])) >= th) bits |= 1u << e;
+                return bits;
+              });
       };
-      int64_t i = threadIdx.x;
-      for (; i + 3 * kTopThreads < nv; i += 4 * kTopThreads) {
+      // Loop bounds are the warp's (its last lane's), so every lane takes
+      // part in every warp-wide step.
+      int64_t i0 = 32 * warp;
+      for (; i0 + 31 + 3 * kTopThreads < nv; i0 += 4 * kTopThreads) {
+        const int64_t i = i0 + lane;
         uint4 va[4], vb[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -705,35 +779,62 @@ __global__ void __launch_bounds__(kTopThreads)
         }
         push_units<4>(vs, va, vb, c);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) visit(va[u], i + u * kTopThreads);
+        for (int u = 0; u < 4; ++u) visit(va[u], i + u * kTopThreads, true);
       }
-      for (; i < nv; i += kTopThreads) {
-        const uint4 va[1] = {ld_stream_v4(a_row + 8 * i)};
-        const uint4 vb[1] = {ld_stream_v4(b_row + 8 * i)};
-        push_units<1>(vs, va, vb, c);
-        visit(va[0], i);
+      for (; i0 < nv; i0 += kTopThreads) {
+        const int64_t u = i0 + lane;
+        const bool valid = u < nv;
+        uint4 va = make_uint4(0u, 0u, 0u, 0u);
+        if (valid) {
+          va = ld_stream_v4(a_row + 8 * u);
+          const uint4 a1[1] = {va};
+          const uint4 b1[1] = {ld_stream_v4(b_row + 8 * u)};
+          push_units<1>(vs, a1, b1, c);
+        }
+        visit(va, u, valid);
       }
       st = vec_stat_final(vs, c);
     } else {
       st = RowStat{{-INFINITY, 0.0f}, {-INFINITY, 0.0f}, 0.0f};
-      for (int64_t v = threadIdx.x; v < V; v += kTopThreads) {
-        const float a = __uint_as_float(static_cast<uint32_t>(a_row[v]) << 16);
-        const float b = __uint_as_float(static_cast<uint32_t>(b_row[v]) << 16);
-        push(st, a, b, c);
-        top_push(top, a, static_cast<int>(v));
+      for (int64_t v0 = 32 * warp; v0 < V; v0 += kTopThreads) {
+        const int64_t v = v0 + lane;
+        const bool valid = v < V;
+        float a = -INFINITY;
+        if (valid) {
+          a = __uint_as_float(static_cast<uint32_t>(a_row[v]) << 16);
+          const float b = __uint_as_float(static_cast<uint32_t>(b_row[v]) << 16);
+          push(st, a, b, c);
+        }
+        offer(valid && a >= thr, a,
+              [&](int src, int, float& x, int& ix) {
+                x = __shfl_sync(kFull, a, src);
+                ix = __shfl_sync(kFull, static_cast<int>(v), src);
+              },
+              [&](float th) { return a >= th ? 1u : 0u; });
+      }
+    }
+    // The warp's K best, lane r holding the r-th: its sorted list.
+    TopList<KM> top;
+    top_init(top);
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+      const float v = __shfl_sync(kFull, lv, j);
+      const int ix = __shfl_sync(kFull, li, j);
+      if (j < K) {
+        top.v[j] = v;
+        top.i[j] = ix;
       }
     }
     // Row statistics and the warps' top-K lists.
     Part mine{st, 0.0f};
     mine = warp_reduce(mine, c);
-    float mv;
-    int mi;
-    top_warp_merge(top, K, mv, mi);
     if (lane == 0) parts[warp] = mine;
-    if (lane < K) {
-      wv[warp][lane] = mv;
-      wi[warp][lane] = mi;
-    }
+#pragma unroll
+    for (int j = 0; j < KM; ++j)
+      if (lane == j && j < K) {
+        wv[warp][j] = top.v[j];
+        wi[warp][j] = top.i[j];
+      }
     __syncthreads();
     if (warp == 0) {
       Part tot = (lane < kWarps) ? parts[lane]
