@@ -7,13 +7,13 @@
 // weights are packed to the per-layer bitwidth when loaded).  The encode is
 // the plain round-to-nearest baseline the reddit excerpt names (RTN).
 //
-// Kernel shape: one warp per 128-weight group.  Lane l holds weights
-// [4l, 4l+4) (one 8-byte load), the min/max are warp reductions, every
-// lane derives the same fp16 scale and zero point, and the 4 codes of a lane
-// form a 4b-bit chunk at stream bit 4b*l.  Lane j < 4b then gathers word j of
-// the group from the (at most five) lanes whose chunks overlap it and stores
-// it, so a group's 4b words leave as one coalesced store.  HBM-bound: 2 bytes
-// read and b/8 + 3/128 bytes written per weight.
+// Kernel shape: eight lanes per 128-weight group, four groups per warp.
+// Lane sl of a group holds weights [16 sl, 16 sl + 16) (two 16-byte loads),
+// the min/max are shuffle reductions inside the eight lanes, and the scale and
+// zero point are formed once per lane for its 16 weights.  The 16 codes of a
+// lane are 16b consecutive stream bits: whole words for even b, half of a
+// lane pair's b words for odd b.  HBM-bound on paper: 2 bytes read and
+// b/8 + 3/128 bytes written per weight.
 //
 // Bit-exactness with the binary32 definition: IEEE division (__fdiv_rn) for
 // the scale and zero point and wherever the reciprocal product could round
@@ -61,20 +61,43 @@ __device__ __forceinline__ float rne_quotient(float w, float s, float r) {
   return k;
 }
 
+// One group per 8 lanes (a warp encodes four groups at once): lane sl of the
+// group holds weights [16 sl, 16 sl + 16).  min / max are shuffle reductions
+// inside the 8 lanes; the scale and zero point are formed once per lane and
+// serve 16 weights.  The 16 codes of a lane are 16b stream bits: for even b
+// whole words (b/2 per lane, stored as they are); for odd b a lane pair
+// joins its 32b bits into b words with one shuffle.
 template <int B>
-__device__ __forceinline__ void encode_group(uint2 raw, int64_t grp, int lane,
-                                             uint32_t* __restrict__ packed,
-                                             uint16_t* __restrict__ scales,
-                                             uint8_t* __restrict__ zeros,
-                                             uint32_t* __restrict__ flags) {
-  const float w[4] = {bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y)};
-  const bool nonfinite =
-      !(isfinite(w[0]) && isfinite(w[1]) && isfinite(w[2]) && isfinite(w[3]));
-  const bool any_nonfinite = __any_sync(kFull, nonfinite);
-
-  // Group statistics: min and max (exact in binary32).
-  const float mn = warp_min(fminf(fminf(w[0], w[1]), fminf(w[2], w[3])));
-  const float mx = warp_max(fmaxf(fmaxf(w[0], w[1]), fmaxf(w[2], w[3])));
+__device__ __forceinline__ void encode_group8(const uint4 (&raw)[2], int64_t grp, bool valid,
+                                              uint32_t* __restrict__ packed,
+                                              uint16_t* __restrict__ scales,
+                                              uint8_t* __restrict__ zeros,
+                                              uint32_t* __restrict__ flags) {
+  const int lane = threadIdx.x & 31;
+  const int sl = lane & 7;
+  const unsigned seg = 0xFFu << (lane & 24);
+  const uint32_t wds[8] = {raw[0].x, raw[0].y, raw[0].z, raw[0].w, raw[1].x, raw[1].y, raw[1].z, raw[1].w};
+  float w[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    w[2 * i] = bf16_lo(wds[i]);
+    w[2 * i + 1] = bf16_hi(wds[i]);
+  }
+  bool nonfinite = false;
+  float mn = w[0], mx = w[0];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    nonfinite |= !isfinite(w[i]);
+    mn = fminf(mn, w[i]);
+    mx = fmaxf(mx, w[i]);
+  }
+  const bool any_nonfinite = (__ballot_sync(kFull, nonfinite) & seg) != 0;
+  // Group statistics: min and max (exact in binary32), inside the 8 lanes.
+#pragma unroll
+  for (int off = 4; off > 0; off >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(kFull, mn, off));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
+  }
 
   // A constant group is widened to include 0.
   float lo = mn, hi = mx;
@@ -101,31 +124,46 @@ __device__ __forceinline__ void encode_group(uint2 raw, int64_t grp, int lane,
   }
   const float s = __half2float(__ushort_as_half(s16));
   const float zf = fminf(fmaxf(rintf(__fdiv_rn(-lo, s)), 0.0f), maxq);
-
   const float r = __frcp_rn(s);
-  uint32_t chunk = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float v = fminf(fmaxf(__fadd_rn(rne_quotient(w[i], s, r), zf), 0.0f), maxq);
-    chunk |= static_cast<uint32_t>(v) << (B * i);
-  }
 
-  // Assemble word j = lane of the group's 4B words from the overlapping chunks.
-  constexpr int kChunkBits = 4 * B;
-  constexpr int kMaxSources = (32 + kChunkBits - 1) / kChunkBits + 1;
-  const int j = lane;
-  const int first = (32 * j) / kChunkBits;
-  uint32_t word = 0;
+  // The lane's 16 codes as a little-endian bit string of 16b bits.
+  constexpr int kLaneWords = (16 * B + 31) / 32;
+  uint32_t words[kLaneWords];
 #pragma unroll
-  for (int i = 0; i < kMaxSources; ++i) {
-    const int src = first + i;
-    const uint32_t v = __shfl_sync(kFull, chunk, src & 31);
-    const int off = kChunkBits * src - 32 * j;  // chunk start relative to word start
-    if (j < kChunkBits && src < 32 && off < 32 && off > -kChunkBits)
-      word |= (off >= 0) ? (v << off) : (v >> (-off));
+  for (int k = 0; k < kLaneWords; ++k) words[k] = 0u;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t q = static_cast<uint32_t>(fminf(fmaxf(__fadd_rn(rne_quotient(w[i], s, r), zf), 0.0f), maxq));
+    const int bit = i * B, wi = bit >> 5, sh = bit & 31;
+    words[wi] |= q << sh;
+    if (sh + B > 32) words[wi + 1] |= q >> (32 - sh);
   }
-  if (j < kChunkBits) packed[grp * kChunkBits + j] = word;
-  if (lane == 0) {
+  uint32_t* out = packed + grp * (4 * B);
+  if constexpr (B % 2 == 0) {
+    if (valid) {
+#pragma unroll
+      for (int k = 0; k < B / 2; ++k) out[sl * (B / 2) + k] = words[k];
+    }
+  } else {
+    // Lane pair (even e, odd o): word k of its b words is
+    // E[k] | O[k - h] << 16 | O[k - h - 1] >> 16, h = (b - 1) / 2.
+    uint32_t other[kLaneWords];
+#pragma unroll
+    for (int k = 0; k < kLaneWords; ++k) other[k] = __shfl_xor_sync(kFull, words[k], 1);
+    const bool odd = sl & 1;
+    constexpr int h = (B - 1) / 2;
+    constexpr int kEven = (B + 1) / 2;  // words the even lane stores
+    auto E = [&](int k) { return (k >= 0 && k < kLaneWords) ? (odd ? other[k] : words[k]) : 0u; };
+    auto O = [&](int k) { return (k >= 0 && k < kLaneWords) ? (odd ? words[k] : other[k]) : 0u; };
+    if (valid) {
+      uint32_t* pw = out + (sl >> 1) * B;
+#pragma unroll
+      for (int k = 0; k < B; ++k) {
+        if ((k < kEven) != odd) pw[k] = E(k) | (O(k - h) << 16) | (O(k - h - 1) >> 16);
+      }
+    }
+  }
+  if (valid && sl == 0) {
     scales[grp] = s16;
     zeros[grp] = static_cast<uint8_t>(zf);
     uint32_t f = (any_nonfinite ? kFlagNonfinite : 0u) | (overflow ? kFlagScaleOverflow : 0u);
@@ -139,19 +177,22 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
                     uint32_t* __restrict__ packed, uint16_t* __restrict__ scales,
                     uint8_t* __restrict__ zeros, uint32_t* __restrict__ flags) {
   const int lane = threadIdx.x & 31;
+  const int sub = lane >> 3, sl = lane & 7;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t base = warp * kUnroll; base < total_groups; base += nwarps * kUnroll) {
-    uint2 raw[kUnroll];
+  for (int64_t base = warp * 4 * kUnroll; base < total_groups; base += nwarps * 4 * kUnroll) {
+    uint4 raw[kUnroll][2];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const int64_t grp = base + u;
-      raw[u] = (grp < total_groups) ? ld_stream_v2(W + grp * kGroup + lane * 4) : make_uint2(0, 0);
+      const int64_t grp = base + 4 * u + sub;
+      const uint16_t* src = W + grp * kGroup + 16 * sl;
+      raw[u][0] = (grp < total_groups) ? ld_stream_v4(src) : make_uint4(0, 0, 0, 0);
+      raw[u][1] = (grp < total_groups) ? ld_stream_v4(src + 8) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const int64_t grp = base + u;
-      if (grp < total_groups) encode_group<B>(raw[u], grp, lane, packed, scales, zeros, flags);
+      const int64_t grp = base + 4 * u + sub;
+      encode_group8<B>(raw[u], grp, grp < total_groups, packed, scales, zeros, flags);
     }
   }
 }
@@ -163,7 +204,7 @@ cudaError_t launch_b(const uint16_t* W, int64_t total_groups, uint32_t* packed,
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t per_block = kWarpsPerBlock * kUnroll;
+  const int64_t per_block = kWarpsPerBlock * 4 * kUnroll;
   int64_t blocks = (total_groups + per_block - 1) / per_block;
   const int64_t cap = static_cast<int64_t>(sms) * 8;  // 8 resident blocks of 256 threads
   if (blocks > cap) blocks = cap;
