@@ -670,12 +670,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 // through L1; the S partial tiles are added in shared memory in warp order
 // (deterministic, no cross-CTA step).
 //
-// For b = 3, 5, 6, 7 (codes cut by word boundaries, the costliest to unpack)
-// the zero point leaves the inner loop: the A pairs are the exact bf16 values
-// 128 + q (q < 128), one more mma per k-step with an all-ones A gives
-// sum_k x over the group, and the group's product is
-// s * (sum (128 + q) x - (128 + z) sum x).  For b = 2, 4, 8 the pairs are
-// (q - z) as above.
+// For b <= 7 the zero point leaves the inner loop: the A pairs are the exact
+// bf16 values 128 + q (q < 128), one more mma per k-step with an all-ones A
+// gives sum_k x over the group, and the group's product is
+// s * (sum (128 + q) x - (128 + z) sum x).  For b = 2 and 4 a pair takes two
+// codes 16 bits apart in one word (one shift, one mask/or) and the
+// activation pairs are permuted to the same k order; b = 3, 5, 6, 7 take
+// consecutive codes.  For b = 8 (q up to 255 is not 128 + q in bf16) the
+// pairs are (q - z) as above.
 // ---------------------------------------------------------------------------
 template <int B>
 __device__ __forceinline__ void lds_unit(const uint8_t* p, uint32_t (&w)[B]) {
@@ -706,9 +708,49 @@ __device__ __forceinline__ uint32_t pair_raw(const uint32_t (&w)[B], int p) {
   } else if constexpr (B == 2) {
     const uint32_t y = __byte_perm(w[p >> 3], 0u, 0x4440 | ((p >> 1) & 3)) * 0x4001u;
     return ((y >> (4 * (p & 1))) & 0x00030003u) | 0x43004300u;
+  } else if constexpr (B == 3 || B == 5) {
+    // The pair's 2b bits t; t * (1 + 2^(16-b)) places the second code at bit
+    // 16 (3b < 17, so the two copies of t do not overlap and the sum is an or).
+    const int bit = 2 * B * p, wi = bit >> 5, sh = bit & 31;
+    const uint32_t x = sh + 2 * B <= 32 ? (w[wi] >> sh) : __funnelshift_r(w[wi], w[wi + 1], sh);
+    const uint32_t t = x & ((1u << (2 * B)) - 1u);
+    constexpr uint32_t mask = ((1u << B) - 1u) * 0x00010001u;
+    return ((t * (1u + (1u << (16 - B)))) & mask) | 0x43004300u;
   } else {
     return dq::code_at<B>(w, 2 * p) | (dq::code_at<B>(w, 2 * p + 1) << 16) | 0x43004300u;
   }
+}
+
+// b = 4 and b = 2: pair p of a unit with its two codes 16 bits apart in one
+// word, as exact bf16 (128 + q, 128 + q'): one shift and one mask/or.  For
+// b = 4, pair p = 4 i + s of word i holds codes (8 i + s, 8 i + s + 4); for
+// b = 2, pair p = 8 i + s holds codes (16 i + s, 16 i + s + 8).  The
+// activation pairs are permuted to match (xpair_nib).
+template <int B>
+__device__ __forceinline__ uint32_t pair_nib(const uint32_t (&w)[B], int p) {
+  static_assert(B == 2 || B == 4, "nibble pairs are for b = 2 and b = 4");
+  if constexpr (B == 4) return ((w[p >> 2] >> (4 * (p & 3))) & 0x000F000Fu) | 0x43004300u;
+  else return ((w[p >> 3] >> (2 * (p & 7))) & 0x00030003u) | 0x43004300u;
+}
+
+__device__ __forceinline__ uint32_t u4_comp(const uint4& v, int c) {
+  return c == 0 ? v.x : c == 1 ? v.y : c == 2 ? v.z : v.w;
+}
+
+// Activation fragments (b0, b1) of k-step j for the pair order of pair_nib:
+// xv holds the thread's 32 consecutive activations, 8 per uint4.
+template <int B>
+__device__ __forceinline__ void xpair_nib(const uint4 (&xv)[4], int j, uint32_t& b0, uint32_t& b1) {
+  uint32_t lo, hi;
+  if constexpr (B == 4) {
+    lo = u4_comp(xv[j >> 1], (j & 1));
+    hi = u4_comp(xv[j >> 1], (j & 1) + 2);
+  } else {
+    lo = u4_comp(xv[2 * (j >> 2)], j & 3);
+    hi = u4_comp(xv[2 * (j >> 2) + 1], j & 3);
+  }
+  b0 = __byte_perm(lo, hi, 0x5410);
+  b1 = __byte_perm(lo, hi, 0x7632);
 }
 
 __device__ __forceinline__ uint32_t ld_ro_u16(const void* p) {
@@ -763,7 +805,8 @@ __device__ __forceinline__ void gemv_tile(const GemvLayer& L, int M, int y_f32, 
   constexpr int kTile = 16 * RT;
   constexpr int kRowG = 16 * B;  // bytes of one row's group
   constexpr int kStage = gemv_stage_bytes<B, RT, GB>();
-  constexpr bool kFold = B == 3 || B == 5 || B == 6 || B == 7;
+  constexpr bool kNib = B == 2 || B == 4;
+  constexpr bool kFold = B != 8;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = lane & 3, q = lane >> 2;
   const int G = K / kGroup;
@@ -802,11 +845,17 @@ __device__ __forceinline__ void gemv_tile(const GemvLayer& L, int M, int y_f32, 
 
   // The first stage's weights go to L2 while the previous kernel finishes;
   // nothing is read into the SM before it has completed.
+  // So do this warp's scales and zeros: lane r < 16 RT takes row r.
   if (ng > 0) {
 #pragma unroll
     for (int rt = 0; rt < RT; ++rt)
 #pragma unroll
       for (int h = 0; h < 2; ++h) asm volatile("prefetch.global.L2 [%0];" ::"l"(wrow[rt][h] + g0 * kRowG));
+    if (lane < kTile) {
+      const int64_t o = static_cast<int64_t>(min(tile0 + lane, N - 1)) * G + g0;
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(scales + o));
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(zeros + o));
+    }
   }
   grid_dependency_wait();
   const int nb = (ng + GB - 1) / GB;
@@ -816,10 +865,27 @@ __device__ __forceinline__ void gemv_tile(const GemvLayer& L, int M, int y_f32, 
     cp_async_commit();
   }
   // This warp's scales and zeros, (scale | zero << 16) per (row, group).
-  for (int idx = lane; idx < kTile * ng; idx += 32) {
-    const int r = idx / ng, gg = idx - r * ng;
-    const int64_t o = static_cast<int64_t>(min(tile0 + r, N - 1)) * G + g0 + gg;
-    szs[r * gmax + gg] = ld_ro_u16(scales + o) | (ld_ro_u8(zeros + o) << 16);
+  // Each lane issues up to kSzBatch loads of each kind before its first
+  // store, so a batch costs one memory latency rather than one per entry.
+  constexpr int kSzBatch = 8;
+  for (int base = 0; base < kTile * ng; base += 32 * kSzBatch) {
+    uint32_t sv[kSzBatch], zv[kSzBatch];
+    int at[kSzBatch];
+#pragma unroll
+    for (int u = 0; u < kSzBatch; ++u) {
+      const int idx = base + 32 * u + lane;
+      at[u] = -1;
+      if (idx < kTile * ng) {
+        const int r = idx / ng, gg = idx - r * ng;
+        const int64_t o = static_cast<int64_t>(min(tile0 + r, N - 1)) * G + g0 + gg;
+        sv[u] = ld_ro_u16(scales + o);
+        zv[u] = ld_ro_u8(zeros + o);
+        at[u] = r * gmax + gg;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kSzBatch; ++u)
+      if (at[u] >= 0) szs[at[u]] = sv[u] | (zv[u] << 16);
   }
   __syncwarp();
 
@@ -883,15 +949,24 @@ __device__ __forceinline__ void gemv_tile(const GemvLayer& L, int M, int y_f32, 
       uint32_t b0[NT], b1[NT];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        b0[nt] = (j & 1) ? xv[nt][j >> 1].z : xv[nt][j >> 1].x;
-        b1[nt] = (j & 1) ? xv[nt][j >> 1].w : xv[nt][j >> 1].y;
+        if constexpr (kNib) {
+          xpair_nib<B>(xv[nt], j, b0[nt], b1[nt]);
+        } else {
+          b0[nt] = (j & 1) ? xv[nt][j >> 1].z : xv[nt][j >> 1].x;
+          b1[nt] = (j & 1) ? xv[nt][j >> 1].w : xv[nt][j >> 1].y;
+        }
         if constexpr (kFold)
           mma_bf16_16816(dsum[nt], 0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u, b0[nt], b1[nt]);
       }
 #pragma unroll
       for (int rt = 0; rt < RT; ++rt) {
         uint32_t a0, a1, a2, a3;
-        if constexpr (kFold) {
+        if constexpr (kNib) {
+          a0 = pair_nib<B>(w[rt][0], 2 * j);
+          a1 = pair_nib<B>(w[rt][1], 2 * j);
+          a2 = pair_nib<B>(w[rt][0], 2 * j + 1);
+          a3 = pair_nib<B>(w[rt][1], 2 * j + 1);
+        } else if constexpr (kFold) {
           a0 = pair_raw<B>(w[rt][0], 2 * j);
           a1 = pair_raw<B>(w[rt][1], 2 * j);
           a2 = pair_raw<B>(w[rt][0], 2 * j + 1);
