@@ -24,8 +24,9 @@ bool encode_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const voi
                           uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
                           uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
-// Decode dequantize-GEMM (M <= 16): dequant to TMEM + tcgen05.mma with the
-// weights as the TMEM operand, persistent stream-K over one CTA per SM.
+// Decode dequantize-GEMM (M <= 16), the SLQ_GEMM_DECODE path: packed W
+// streamed by TMA, dequantized in registers into mma.sync A fragments,
+// persistent stream-K over two CTAs per SM with a deterministic fixup.
 // `workspace` holds the split tiles' counters and partial sums
 // (gemm_decode_workspace_bytes; zero-filled counters on entry and exit).
 cudaError_t launch_gemm_decode(const uint16_t* X, int64_t M, int64_t N, int64_t K, int bits,
