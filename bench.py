@@ -282,10 +282,8 @@ def run_slq(args, rank, world, local_rank):
     ms_total = t0.elapsed_time(t1)
     clk = clocks.stop()
     ms_step = ms_total / (args.steps * reps)
+    ms_step = max_over_ranks(ms_step, dist, dev)
     if dist:
-        t = torch.tensor([ms_step], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
         dist.barrier()
 
     value = world * 3 * BLOCK_BYTES / (ms_step * 1e-3) / 1e9  # GB/s, whole job
@@ -350,10 +348,7 @@ def run_slq(args, rank, world, local_rank):
     e1.record(stream)
     e1.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if dist:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
     e2e_value = world * 3 * BLOCK_BYTES / (e2e_ms * 1e-3) / 1e9
 
     rows = {}
@@ -414,6 +409,17 @@ def run_slq(args, rank, world, local_rank):
         if cpu is not None:
             out["cpu_baseline"] = cpu
     return out
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """The largest `value` over all ranks (a replicated job takes as long as
+    its slowest rank); `value` itself when there is no process group."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def time_ms(torch, stream, fn, iters, warm=2):
