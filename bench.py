@@ -495,22 +495,57 @@ def other_rows(args, slq, synth, torch, dev, stream, hbm_peak, tc_peak, rank):
         tf = 2 * M * N * K / (ms * 1e-3) / 1e12
         pre[f"{name}_M{M}"] = {"TFLOPs": round(tf, 1), "frac_tensor": round(tf / tc_peak, 3), "us": round(ms * 1e3, 1)}
         del qw, Xp, Yp
+    # The sizes reported only, M = 64 and 256 on 8192^2 (memory-bound for
+    # b >= 3): weights rotated over more than L2, launches replayed from a graph.
+    N = K = 8192
+    for b in (2, 4, 8):
+        nrot = max(2, int(np.ceil(4 * L2_BYTES / weight_bytes(N, K, b))))
+        qws = [slq.quantize(synth.weights_torch(N, K, seed=920 + b + 10 * r, device=dev), b) for r in range(nrot)]
+        for M in (64, 256):
+            Xp = synth.activations_torch(M, K, seed=921, device=dev)
+            Yp = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            slq.gemm(Xp, qws[0], out=Yp, stream=stream)
+            stream.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for r in range(nrot):
+                    slq.gemm(Xp, qws[r], out=Yp, stream=stream)
+            ms = time_ms(torch, stream, g.replay, 10) / nrot
+            gbps = weight_bytes(N, K, b) / (ms * 1e-3) / 1e9
+            tf = 2 * M * N * K / (ms * 1e-3) / 1e12
+            pre[f"sweep8192_b{b}_M{M}"] = {"GBps": round(gbps, 1), "frac_hbm": round(gbps / hbm_peak, 3),
+                                           "TFLOPs": round(tf, 1), "frac_tensor": round(tf / tc_peak, 3),
+                                           "us": round(ms * 1e3, 1)}
+            del g, Xp, Yp
+        del qws
+    # The Llama-3.3-70B-shaped block (683 MB of packed weights, more than
+    # L2) at M = 1, 16, 64 and 2048: seven launches per step.
     llama = [(8192, 8192, 7), (1024, 8192, 8), (1024, 8192, 8), (8192, 8192, 7), (28672, 8192, 6),
              (28672, 8192, 6), (8192, 28672, 6)]
-    M = 2048
     qws = [slq.quantize(synth.weights_torch(N, K, seed=950 + i, device=dev), b) for i, (N, K, b) in enumerate(llama)]
-    Xs = [synth.activations_torch(M, K, seed=960 + i, device=dev) for i, (N, K, b) in enumerate(llama)]
-    Ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for (N, K, b) in llama]
+    wbytes = sum(weight_bytes(N, K, b) for (N, K, b) in llama)
+    for M in (1, 16, 64, 2048):
+        Xs = [synth.activations_torch(M, K, seed=960 + i, device=dev) for i, (N, K, b) in enumerate(llama)]
+        Ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for (N, K, b) in llama]
 
-    def block():
-        for x, q, y in zip(Xs, qws, Ys):
-            slq.gemm(x, q, out=y, stream=stream)
+        def block():
+            for x, q, y in zip(Xs, qws, Ys):
+                slq.gemm(x, q, out=y, stream=stream)
 
-    ms = time_ms(torch, stream, block, 5)
-    flops = sum(2 * M * N * K for (N, K, b) in llama)
-    tf = flops / (ms * 1e-3) / 1e12
-    pre["llama70b_block_M2048"] = {"TFLOPs": round(tf, 1), "frac_tensor": round(tf / tc_peak, 3), "us": round(ms * 1e3, 1)}
-    del qws, Xs, Ys
+        block()
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            block()
+        ms = time_ms(torch, stream, g.replay, 5)
+        flops = sum(2 * M * N * K for (N, K, b) in llama)
+        tf = flops / (ms * 1e-3) / 1e12
+        gbps = wbytes / (ms * 1e-3) / 1e9
+        pre[f"llama70b_block_M{M}"] = {"GBps": round(gbps, 1), "frac_hbm": round(gbps / hbm_peak, 3),
+                                       "TFLOPs": round(tf, 1), "frac_tensor": round(tf / tc_peak, 3),
+                                       "us": round(ms * 1e3, 1)}
+        del g, Xs, Ys
+    del qws
     rows["tiled_prefill"] = pre
 
     # EAR / KL over [4096 x 151936] bf16 logits, tau 1.0 and 0.7.
