@@ -70,6 +70,8 @@ def _load():
         lib.oracle_ear_kl.restype = ctypes.c_int
         lib.oracle_ear_kl_topk.argtypes = [P, P, P, I64, I64, I64, ctypes.c_double, P, P, P]
         lib.oracle_ear_kl_topk.restype = ctypes.c_int
+        lib.oracle_grid_noise.argtypes = [P, I64, I64, ctypes.c_int, P, P, P]
+        lib.oracle_grid_noise.restype = ctypes.c_int
         _lib = lib
         return lib
 
@@ -192,3 +194,20 @@ def ear_kl_topk(a_bf16, b_bf16, k: int, tau: float, rows=None):
     if rc != 0:
         raise ValueError("oracle_ear_kl_topk rejected its arguments")
     return ear, kl, top
+
+
+def grid_noise(w_bf16, bits: int):
+    """Per-group (gamma, sse_asym, sse_sym), each [N, K/128] binary64: the
+    gamma^2-law ablation of an asymmetric grid over [min, max] against a
+    symmetric grid over [-max|w|, max|w|] (see oracle_grid_noise)."""
+    w = _u16(w_bf16)
+    assert w.ndim == 2
+    N, K = w.shape
+    G = K // 128
+    gamma = np.empty((N, G), dtype=np.float64)
+    sse_a = np.empty((N, G), dtype=np.float64)
+    sse_s = np.empty((N, G), dtype=np.float64)
+    rc = _load().oracle_grid_noise(_ptr(w), N, K, int(bits), _ptr(gamma), _ptr(sse_a), _ptr(sse_s))
+    if rc != 0:
+        raise ValueError("oracle_grid_noise rejected its arguments")
+    return gamma, sse_a, sse_s

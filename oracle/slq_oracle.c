@@ -405,3 +405,56 @@ int oracle_ear_kl_topk(const uint16_t *a_bf16, const uint16_t *b_bf16,
   free(sel);
   return 0;
 }
+
+
+/* ------------------------------------------------------------------------
+ * Grid noise of the symmetric-vs-asymmetric ablation.  The pages' gamma^2
+ * law says a symmetric grid over [-M, M] has gamma^2 = (2M / R)^2 times the
+ * noise variance of an asymmetric grid over [lo, hi], because its step is
+ * gamma times larger and rounding noise scales with the step squared.  Per
+ * group this computes gamma and the squared reconstruction error of each
+ * grid, nearest point by rounding the binary64 position (w - start) / step
+ * (ties go to the even index; either neighbour gives the same error).
+ * ------------------------------------------------------------------------ */
+static double grid_sse(const double *w, int n, double start, double step, int levels) {
+  double sse = 0.0;
+  for (int k = 0; k < n; ++k) {
+    double r;
+    if (step == 0.0) {
+      r = start;
+    } else {
+      double i = nearbyint((w[k] - start) / step);
+      if (i < 0.0) i = 0.0;
+      if (i > (double)levels) i = (double)levels;
+      r = start + i * step;
+    }
+    double e = w[k] - r;
+    sse += e * e;
+  }
+  return sse;
+}
+
+int oracle_grid_noise(const uint16_t *w_bf16, int64_t N, int64_t K, int bits,
+                      double *gamma, double *sse_asym, double *sse_sym) {
+  if (N < 0 || K < GROUP || K % GROUP || bits < 2 || bits > 8) return -1;
+  const int levels = (1 << bits) - 1;
+  const int64_t G = K / GROUP;
+  double w[GROUP];
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t g = 0; g < G; ++g) {
+      double lo = 0.0, hi = 0.0, m = 0.0;
+      for (int k = 0; k < GROUP; ++k) {
+        w[k] = (double)oracle_bf16_to_f32(w_bf16[n * K + g * GROUP + k]);
+        if (k == 0 || w[k] < lo) lo = w[k];
+        if (k == 0 || w[k] > hi) hi = w[k];
+        if (fabs(w[k]) > m) m = fabs(w[k]);
+      }
+      const double range = hi - lo;
+      const int64_t o = n * G + g;
+      gamma[o] = range > 0.0 ? 2.0 * m / range : 1.0;
+      sse_asym[o] = grid_sse(w, GROUP, lo, range / levels, levels);
+      sse_sym[o] = grid_sse(w, GROUP, -m, 2.0 * m / levels, levels);
+    }
+  }
+  return 0;
+}

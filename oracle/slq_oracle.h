@@ -85,6 +85,21 @@ int oracle_ear_kl_topk(const uint16_t *a_bf16, const uint16_t *b_bf16,
                        const int64_t *rows, int64_t n_rows, int64_t V, int64_t K,
                        double tau, double *ear, double *kl, int64_t *top);
 
+/* Per-group grid noise for the symmetric-vs-asymmetric ablation (the gamma^2
+ * variance law: wispaper.ai blog, section on the gamma^2 law; gist.science
+ * summary, Methodology section 1).  For each 128-group g of row n of W (bf16
+ * bits, [N, K], K % 128 == 0), with lo = min w, hi = max w, M = max |w|,
+ * R = hi - lo, and L = 2^b - 1 intervals:
+ *   gamma[n, g]    = 2M / R (1 when R == 0);
+ *   sse_asym[n, g] = sum over the group of (w - nearest point of the grid
+ *                    lo + i R / L)^2, i = 0..L;
+ *   sse_sym[n, g]  = the same for the grid -M + i 2M / L.
+ * Both grids in binary64 without scale rounding: this measures the grids
+ * the law compares, not the stored format.  Non-finite weights give
+ * non-finite results.  Returns 0, or -1 on an invalid argument. */
+int oracle_grid_noise(const uint16_t *w_bf16, int64_t N, int64_t K, int bits,
+                      double *gamma, double *sse_asym, double *sse_sym);
+
 #ifdef __cplusplus
 }
 #endif
