@@ -20,7 +20,10 @@
  *   - the Expected Acceptance Rate EAR = sum_v min(p_v, q_v) and KL(p || q)
  *     between two softmaxed logit rows (gist.science summary, "Methodology"
  *     section 2 "Fidelity Metrics"; reddit abstract: EAR is the maximum
- *     token-agreement probability under optimal coupling).
+ *     token-agreement probability under optimal coupling);
+ *   - the per-group noise of a symmetric against an asymmetric grid, the
+ *     ablation behind the gamma^2 variance law (wispaper.ai blog, section on
+ *     the gamma^2 law; gist.science summary, "Methodology" section 1).
  *
  * Precision: encode decisions in IEEE binary32 (the library's format
  * definition fixes fp32 for scale, zero and code); dequantize, GEMM and
