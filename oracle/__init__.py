@@ -70,6 +70,8 @@ def _load():
         lib.oracle_ear_kl.restype = ctypes.c_int
         lib.oracle_ear_kl_topk.argtypes = [P, P, P, I64, I64, I64, ctypes.c_double, P, P, P]
         lib.oracle_ear_kl_topk.restype = ctypes.c_int
+        lib.oracle_gptq.argtypes = [P, I64, I64, ctypes.c_int, P, I64, ctypes.c_double, P, P, P, P]
+        lib.oracle_gptq.restype = ctypes.c_int
         lib.oracle_grid_noise.argtypes = [P, I64, I64, ctypes.c_int, P, P, P]
         lib.oracle_grid_noise.restype = ctypes.c_int
         _lib = lib
@@ -211,3 +213,21 @@ def grid_noise(w_bf16, bits: int):
     if rc != 0:
         raise ValueError("oracle_grid_noise rejected its arguments")
     return gamma, sse_a, sse_s
+
+
+def gptq(w_bf16: np.ndarray, x_bf16: np.ndarray, bits: int, damp: float = 0.01):
+    """GPTQ encode of bf16 W [N, K] with calibration rows X [T, K] (bf16 bits):
+    (packed, scales, zeros, flags) in the format of quantize()."""
+    w = _u16(w_bf16)
+    x = _u16(x_bf16)
+    assert w.ndim == 2 and x.ndim == 2 and x.shape[1] == w.shape[1]
+    N, K = w.shape
+    packed = np.zeros((N, K * bits // 32), dtype=np.uint32)
+    scales = np.zeros((N, K // 128), dtype=np.uint16)
+    zeros = np.zeros((N, K // 128), dtype=np.uint8)
+    flags = ctypes.c_uint32(0)
+    rc = _load().oracle_gptq(_ptr(w), N, K, int(bits), _ptr(x), x.shape[0], float(damp),
+                             _ptr(packed), _ptr(scales), _ptr(zeros), ctypes.byref(flags))
+    if rc != 0:
+        raise ValueError(f"oracle_gptq failed ({rc})")
+    return packed, scales, zeros, int(flags.value)

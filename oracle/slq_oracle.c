@@ -126,14 +126,11 @@ uint32_t oracle_code_at(const uint32_t *packed, int64_t K, int bits, int64_t n,
  *   scale = (max - min) / (2^b - 1), zero = clamp(rne(-min / scale)),
  *   q = clamp(rne(w / scale) + zero), codes in [0, 2^b - 1].
  */
-static void quantize_group(const uint16_t *src, int bits, uint16_t *s16_out,
-                           uint8_t *z_out, uint32_t *codes, uint32_t *flags) {
-  float w[GROUP];
+static void group_params(const float *w, int bits, uint16_t *s16_out, float *z_out,
+                         uint32_t *flags) {
   int nonfinite = 0;
-  for (int k = 0; k < GROUP; ++k) {
-    w[k] = oracle_bf16_to_f32(src[k]);
+  for (int k = 0; k < GROUP; ++k)
     if (!isfinite(w[k])) nonfinite = 1;
-  }
   if (nonfinite && flags) *flags |= ORACLE_FLAG_NONFINITE;
 
   /* Group statistics: min and max in binary32 (exact). */
@@ -174,16 +171,29 @@ static void quantize_group(const uint16_t *src, int bits, uint16_t *s16_out,
   float zf = rintf(-lo / s);
   if (zf != zf || zf < 0.0f) zf = 0.0f;
   if (zf > maxq) zf = maxq;
-
-  /* Codes: rne(w / scale) + zero, clamped to the code range.  The sum is
-   * taken in binary32: it is exact whenever the result is inside the range. */
-  for (int k = 0; k < GROUP; ++k) {
-    float v = rintf(w[k] / s) + zf;
-    if (v != v || v < 0.0f) v = 0.0f;
-    if (v > maxq) v = maxq;
-    codes[k] = (uint32_t)v;
-  }
   *s16_out = s16;
+  *z_out = zf;
+}
+
+/* Code of one weight: rne(w / scale) + zero, clamped to the code range.  The
+ * sum is taken in binary32: it is exact whenever the result is inside the
+ * range. */
+static uint32_t encode_one(float w, float s, float zf, int bits) {
+  const float maxq = (float)((1 << bits) - 1);
+  float v = rintf(w / s) + zf;
+  if (v != v || v < 0.0f) v = 0.0f;
+  if (v > maxq) v = maxq;
+  return (uint32_t)v;
+}
+
+static void quantize_group(const uint16_t *src, int bits, uint16_t *s16_out,
+                           uint8_t *z_out, uint32_t *codes, uint32_t *flags) {
+  float w[GROUP];
+  for (int k = 0; k < GROUP; ++k) w[k] = oracle_bf16_to_f32(src[k]);
+  float zf;
+  group_params(w, bits, s16_out, &zf, flags);
+  const float s = (float)oracle_f16_to_f64(*s16_out);
+  for (int k = 0; k < GROUP; ++k) codes[k] = encode_one(w[k], s, zf, bits);
   *z_out = (uint8_t)zf;
 }
 
@@ -205,6 +215,139 @@ int oracle_quantize(const uint16_t *w_bf16, int64_t N, int64_t K, int bits,
     }
   }
   return 0;
+}
+
+/* ---------------------------------------------------------------------- */
+/* GPTQ with this format's quantizer.                                      */
+/* ---------------------------------------------------------------------- */
+
+/* In-place lower Cholesky factor of the n x n row-major matrix a (a = L L^T);
+ * the upper triangle is zeroed.  Returns -1 if a is not positive definite. */
+static int cholesky_lower(double *a, int64_t n) {
+  for (int64_t j = 0; j < n; ++j) {
+    double d = a[j * n + j];
+    for (int64_t k = 0; k < j; ++k) d -= a[j * n + k] * a[j * n + k];
+    if (!(d > 0.0)) return -1;
+    d = sqrt(d);
+    a[j * n + j] = d;
+    for (int64_t i = j + 1; i < n; ++i) {
+      double v = a[i * n + j];
+      for (int64_t k = 0; k < j; ++k) v -= a[i * n + k] * a[j * n + k];
+      a[i * n + j] = v / d;
+    }
+    for (int64_t k = j + 1; k < n; ++k) a[j * n + k] = 0.0;
+  }
+  return 0;
+}
+
+/*
+ * GPTQ (Frantar et al., "GPTQ: Accurate Post-Training Quantization for
+ * Generative Pre-trained Transformers"): the encoder the pages run for every
+ * layer at every b (GitHub README, "Pipeline" and "1. Quantize": layer-wise
+ * GPTQ, asymmetric INT, group size 128).  Each row of W is encoded column by
+ * column; after a column is fixed, the error it leaves is spread over the
+ * row's later columns so as to minimize the change of X W^T on the
+ * calibration rows X.  Readings where the pages are silent:
+ *   - H = X^T X in binary64 (the usual factor 2/T does not change the
+ *     result); a column with H_kk = 0 (an input that is always zero) gets
+ *     H_kk = 1 and its weights set to 0;
+ *   - damping H += damp * mean(diag H) * I;
+ *   - columns in their natural order (no activation ordering);
+ *   - a group's scale and zero come from the group's current, already
+ *     updated weights when its first column is reached, by the RTN rules
+ *     above;
+ *   - the weights are carried in binary64 and rounded to binary32 for the
+ *     encode decision;
+ *   - with U the upper Cholesky factor of H^-1 (H^-1 = U^T U), fixing column
+ *     k with dequantized value d moves every later column j of the row by
+ *     -(w_k - d) / U_kk * U_kj.
+ * x_bf16: [T, K] calibration rows.  Returns 0; -1 on an invalid argument;
+ * -2 if the damped H is not positive definite or memory runs out.
+ */
+int oracle_gptq(const uint16_t *w_bf16, int64_t N, int64_t K, int bits,
+                const uint16_t *x_bf16, int64_t T, double damp, uint32_t *packed,
+                uint16_t *scales_f16, uint8_t *zeros, uint32_t *flags) {
+  if (bits < 2 || bits > 8 || N < 0 || K < GROUP || K % GROUP != 0 || T < 1 ||
+      !(damp >= 0.0) || isinf(damp))
+    return -1;
+  const int64_t G = K / GROUP;
+  const int64_t words_per_row = K * bits / 32;
+  double *h = (double *)calloc((size_t)(K * K), sizeof(double));
+  double *inv = (double *)calloc((size_t)(K * K), sizeof(double));
+  double *x = (double *)malloc((size_t)K * sizeof(double));
+  double *w = (double *)malloc((size_t)K * sizeof(double));
+  unsigned char *dead = (unsigned char *)calloc((size_t)K, 1);
+  int rc = -2;
+  if (!h || !inv || !x || !w || !dead) goto done;
+
+  /* H = X^T X. */
+  for (int64_t t = 0; t < T; ++t) {
+    for (int64_t k = 0; k < K; ++k) x[k] = (double)oracle_bf16_to_f32(x_bf16[t * K + k]);
+    for (int64_t i = 0; i < K; ++i)
+      for (int64_t j = 0; j <= i; ++j) h[i * K + j] += x[i] * x[j];
+  }
+  for (int64_t i = 0; i < K; ++i)
+    for (int64_t j = 0; j < i; ++j) h[j * K + i] = h[i * K + j];
+  double mean = 0.0;
+  for (int64_t k = 0; k < K; ++k) {
+    if (h[k * K + k] == 0.0) {
+      h[k * K + k] = 1.0;
+      dead[k] = 1;
+    }
+    mean += h[k * K + k];
+  }
+  mean /= (double)K;
+  for (int64_t k = 0; k < K; ++k) h[k * K + k] += damp * mean;
+
+  /* H^-1 = L^-T L^-1 from H = L L^T, then U^T = the lower factor of H^-1. */
+  if (cholesky_lower(h, K) != 0) goto done;
+  for (int64_t c = 0; c < K; ++c) { /* column c of L^-1 by forward substitution */
+    for (int64_t i = 0; i < K; ++i) {
+      double v = (i == c) ? 1.0 : 0.0;
+      for (int64_t k = c; k < i; ++k) v -= h[i * K + k] * inv[k * K + c];
+      inv[i * K + c] = (i < c) ? 0.0 : v / h[i * K + i];
+    }
+  }
+  for (int64_t i = 0; i < K; ++i) /* h := (L^-1)^T L^-1, i.e. H^-1 */
+    for (int64_t j = 0; j < K; ++j) {
+      double v = 0.0;
+      for (int64_t k = (i > j ? i : j); k < K; ++k) v += inv[k * K + i] * inv[k * K + j];
+      h[i * K + j] = v;
+    }
+  if (cholesky_lower(h, K) != 0) goto done; /* h = U^T: U_kj = h[j][k] */
+
+  memset(packed, 0, (size_t)(N * words_per_row) * sizeof(uint32_t));
+  for (int64_t n = 0; n < N; ++n) {
+    uint32_t *row_words = packed + n * words_per_row;
+    for (int64_t k = 0; k < K; ++k)
+      w[k] = dead[k] ? 0.0 : (double)oracle_bf16_to_f32(w_bf16[n * K + k]);
+    uint16_t s16 = 0;
+    float s = 0.0f, zf = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+      if (k % GROUP == 0) {
+        float wg[GROUP];
+        for (int j = 0; j < GROUP; ++j) wg[j] = (float)w[k + j];
+        group_params(wg, bits, &s16, &zf, flags);
+        s = (float)oracle_f16_to_f64(s16);
+        scales_f16[n * G + k / GROUP] = s16;
+        zeros[n * G + k / GROUP] = (uint8_t)zf;
+      }
+      const uint32_t q = encode_one((float)w[k], s, zf, bits);
+      put_code(row_words, k * bits, bits, q);
+      const double d = oracle_f16_to_f64(s16) * ((double)q - (double)zf);
+      const double u_kk = h[k * K + k];
+      const double e = (w[k] - d) / u_kk;
+      for (int64_t j = k + 1; j < K; ++j) w[j] -= e * h[j * K + k];
+    }
+  }
+  rc = 0;
+done:
+  free(h);
+  free(inv);
+  free(x);
+  free(w);
+  free(dead);
+  return rc;
 }
 
 /* ---------------------------------------------------------------------- */

@@ -57,6 +57,15 @@ int oracle_quantize(const uint16_t *w_bf16, int64_t N, int64_t K, int bits,
                     uint32_t *packed, uint16_t *scales_f16, uint8_t *zeros,
                     uint32_t *flags);
 
+/* GPTQ encode of W (bf16 bits, [N, K]) to b bits in the same format as
+ * oracle_quantize, with calibration rows x (bf16 bits, [T, K]) and relative
+ * damping damp (readings in slq_oracle.c).  flags may be NULL.  Returns 0,
+ * -1 on an invalid argument, -2 if the damped X^T X is singular or memory
+ * runs out. */
+int oracle_gptq(const uint16_t *w_bf16, int64_t N, int64_t K, int bits,
+                const uint16_t *x_bf16, int64_t T, double damp, uint32_t *packed,
+                uint16_t *scales_f16, uint8_t *zeros, uint32_t *flags);
+
 /* Read code k of row n back out of the packed stream. */
 uint32_t oracle_code_at(const uint32_t *packed, int64_t K, int bits,
                         int64_t n, int64_t k);
