@@ -21,6 +21,8 @@
  *     between two softmaxed logit rows (gist.science summary, "Methodology"
  *     section 2 "Fidelity Metrics"; reddit abstract: EAR is the maximum
  *     token-agreement probability under optimal coupling);
+ *   - GPTQ with this format's quantizer, the encoder the pages run for every
+ *     layer at every b (GitHub README, "Pipeline" and "1. Quantize");
  *   - the per-group noise of a symmetric against an asymmetric grid, the
  *     ablation behind the gamma^2 variance law (wispaper.ai blog, section on
  *     the gamma^2 law; gist.science summary, "Methodology" section 1).
