@@ -6,8 +6,9 @@ CPU-baseline/reference leg may import it; the product path
 (``weight_only_mixed_b200``) never does, and the two share no code.
 
 The arithmetic lives in ``slq_oracle.c`` (plain C, binary32 encode decisions,
-binary64 dequantize/GEMM/EAR/KL); this module only compiles it with gcc and
-marshals numpy arrays through ctypes.
+binary64 dequantize/GEMM/EAR/KL, GPTQ error feedback and grid-noise sums);
+this module only compiles it with gcc and marshals numpy arrays through
+ctypes.
 """
 from __future__ import annotations
 
