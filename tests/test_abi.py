@@ -1,6 +1,7 @@
 """Host-side checks of the C ABI that need no GPU.
 
-  * libslq.so loads and exports every function include/slq.h declares;
+  * libslq.so loads and exports every function include/slq.h declares, and
+    the binding gives each one its ctypes signature;
   * the header carries no torch or CUDA types in its signatures;
   * argument validation rejects bad calls with SLQ_ERR_INVALID_ARGUMENT
     before touching CUDA (fake, never-dereferenced pointers are used);
@@ -29,6 +30,13 @@ def test_every_declared_symbol_is_exported():
                          text=True, check=True).stdout
     exported = set(re.findall(r"\bT (slq_\w+)", out))
     assert set(names) <= exported
+
+
+def test_binding_declares_every_signature():
+    # Without argtypes ctypes passes Python ints as C int, which would cut
+    # 64-bit sizes and pointers; every declared function gets its signature.
+    for n in slq.declared_symbols():
+        assert getattr(L, n).argtypes is not None, n
 
 
 def test_header_is_plain_c():
