@@ -97,9 +97,8 @@ slq_gemm_path slq_gemm_select(int64_t M, int64_t N, int64_t K, int bits);
 /* Bytes of device workspace the SLQ_GEMM_DECODE kernel needs for
  * Y[M, N] = X[M, K] W[N, K]^T on the CURRENT device (it splits the layer over
  * that device's SMs); 0 when it needs none (every row tile falls in one CTA)
- * and for M > 16.  The kernels slq_gemm selects (GEMV, TILED) need no
- * workspace, so a buffer of this size serves every path.  Returns 0 for
- * invalid arguments.
+ * and for M > 16.  Only slq_gemm_ex with SLQ_GEMM_DECODE takes a workspace.
+ * Returns 0 for invalid arguments.
  *
  * Workspace rules: device memory owned by the caller, 256-byte aligned, not
  * overlapping any other argument.  Its first 64 KiB hold per-row-tile
@@ -160,21 +159,22 @@ slq_status slq_quantize(const void *W_bf16, int64_t N, int64_t K, int bits,
  *             same kernel writes with SLQ_DTYPE_F32: the order of every sum is
  *             fixed by the sizes and the device, never by timing, so repeated
  *             calls give identical bits.
- * workspace, workspace_bytes   at least slq_gemm_workspace_bytes(M, N, K,
- *             bits) bytes under the workspace rules above; may be NULL / 0
- *             when that is 0.  SLQ_ERR_INVALID_ARGUMENT if too small.
  * flags       device uint32 or NULL; SLQ_FLAG_TIMEOUT.
+ *
+ * The kernels this call selects (SLQ_GEMM_GEMV for M <= 16, SLQ_GEMM_TILED
+ * above) use no memory beyond their arguments: there is no workspace.
  */
 slq_status slq_gemm(const void *X_bf16, int64_t M, int64_t N, int64_t K,
                     int bits, const uint32_t *packed, const void *scales_f16,
                     const uint8_t *zeros, void *Y, slq_dtype y_dtype,
-                    void *workspace, size_t workspace_bytes, uint32_t *flags,
-                    void *stream);
+                    uint32_t *flags, void *stream);
 
 /* slq_gemm with an explicit kernel choice (SLQ_GEMM_DECODE and SLQ_GEMM_GEMV
- * need M <= 16; only SLQ_GEMM_DECODE needs a workspace, of
- * slq_gemm_workspace_bytes bytes, and takes N <= 2097152).  Same arguments
- * and results otherwise. */
+ * need M <= 16).  Only SLQ_GEMM_DECODE needs a workspace, of
+ * slq_gemm_workspace_bytes bytes under the workspace rules above, and takes
+ * N <= 2097152; `workspace` may be NULL / 0 for every other path and when
+ * that size is 0 (SLQ_ERR_INVALID_ARGUMENT if too small).  Same arguments and
+ * results otherwise. */
 slq_status slq_gemm_ex(const void *X_bf16, int64_t M, int64_t N, int64_t K,
                        int bits, const uint32_t *packed,
                        const void *scales_f16, const uint8_t *zeros, void *Y,
@@ -246,7 +246,9 @@ int slq_gemm_group_max(void);
  * same time on the GPU (different streams, or several host threads) race on
  * it and give wrong results; issue them one after another on one stream.
  * The first call on a device looks up the array's device address (with that
- * device current); make that first call before any stream capture.
+ * device current), and so does the first call after the device was reset
+ * (cudaDeviceReset gives it a new copy of the array); make such a call before
+ * any stream capture.
  */
 #define SLQ_DECODE_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
 

@@ -108,6 +108,21 @@ def test_gemm_validation():
     assert _g(M=0) == slq.SLQ_OK and _g(N=0) == slq.SLQ_OK
 
 
+def test_slq_gemm_takes_no_workspace():
+    # slq_gemm(X, M, N, K, bits, packed, scales, zeros, Y, y_dtype, flags, stream):
+    # the kernels it selects use no memory beyond their arguments.
+    def g(M=4, N=8, K=256, bits=4, X=FAKE, Y=FAKE + (4 << 24), dtype=0):
+        return L.slq_gemm(X, M, N, K, bits, FAKE + (1 << 24), FAKE + (2 << 24), FAKE + (3 << 24), Y,
+                          dtype, None, None)
+    assert len(L.slq_gemm.argtypes) == 12
+    for bad in [dict(bits=9), dict(K=100), dict(X=None), dict(Y=FAKE + 16), dict(dtype=2)]:
+        assert g(**bad) == slq.SLQ_ERR_INVALID_ARGUMENT, bad
+    assert g(M=0) == slq.SLQ_OK
+    assert g() in (slq.SLQ_OK, slq.SLQ_ERR_UNSUPPORTED_DEVICE)
+    assert g(M=300, N=4096, K=4096, X=FAKE, Y=FAKE + (8 << 24)) in (slq.SLQ_OK,
+                                                                      slq.SLQ_ERR_UNSUPPORTED_DEVICE)
+
+
 def test_gemm_workspace_rules():
     # A layer whose row tiles are split over several CTAs needs a workspace.
     M, N, K, b = 4, 4096, 4096, 4

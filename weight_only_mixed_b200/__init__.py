@@ -71,7 +71,7 @@ _lib.slq_quantize.restype = _I
 _SZ = ctypes.c_size_t
 _lib.slq_gemm_workspace_bytes.argtypes = [_I64, _I64, _I64, _I]
 _lib.slq_gemm_workspace_bytes.restype = _SZ
-_lib.slq_gemm.argtypes = [_P, _I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _P, _SZ, _P, _P]
+_lib.slq_gemm.argtypes = [_P, _I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _P, _P]
 _lib.slq_gemm.restype = _I
 _lib.slq_gemm_ex.argtypes = [_P, _I64, _I64, _I64, _I, _P, _P, _P, _P, _I, _I, _P, _SZ, _P, _P]
 _lib.slq_gemm_ex.restype = _I

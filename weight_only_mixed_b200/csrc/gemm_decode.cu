@@ -1147,17 +1147,9 @@ cudaError_t launch_cfg(const uint16_t* X, int M, int N, int K, const uint32_t* p
                             static_cast<uint64_t>(K) * B / 32, static_cast<uint64_t>(N),
                             static_cast<uint64_t>(K) * B / 8, 4 * B * GS, kRows, swz))
     return cudaErrorInvalidValue;
-  static bool attr_set = false;  // per template instance
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_decode_kernel<B, NT, GS>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(gemm_decode_kernel<B, NT, GS>,
-                             cudaFuncAttributePreferredSharedMemoryCarveout,
-                             static_cast<int>(cudaSharedmemCarveoutMaxShared));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static SmemAttr smem_attr;  // per template instance
+  const cudaError_t ea = smem_attr.ensure(gemm_decode_kernel<B, NT, GS>, C::kSmem);
+  if (ea != cudaSuccess) return ea;
   const Split sp = make_split(N, K, GS, resident_ctas());
   int* counters = static_cast<int*>(workspace);
   float* partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes);
@@ -1237,13 +1229,9 @@ cudaError_t launch_gemv_cfg(const uint16_t* X, int M, int N, int K, const uint32
   const size_t partb = static_cast<size_t>(S) * 16 * RT * (8 * NT + 1) * 4;
   const size_t smem = (rings + szb) > partb ? rings + szb : partb;
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
-  static int attr_bytes = 0;  // per template instance: the largest size set so far
-  if (static_cast<int>(smem) > attr_bytes) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    attr_bytes = static_cast<int>(smem);
-  }
+  static SmemAttr smem_attr;  // per template instance
+  const cudaError_t ea = smem_attr.ensure(kern, static_cast<int>(smem));
+  if (ea != cudaSuccess) return ea;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>((N + 16 * RT - 1) / (16 * RT)), 1, 1);
   cfg.blockDim = dim3(32 * S, 1, 1);
@@ -1303,7 +1291,8 @@ cudaError_t launch_gemv_b(const uint16_t* X, int M, int N, int K, const uint32_t
 
 cudaError_t launch_gemm_gemv(const uint16_t* X, int64_t M, int64_t N, int64_t K, int bits,
                              const uint32_t* packed, const uint16_t* scales, const uint8_t* zeros,
-                             void* Y, bool y_f32, cudaStream_t stream) {
+                             void* Y, bool y_f32, uint32_t* flags, cudaStream_t stream) {
+  (void)flags;  // the GEMV kernel has no bounded waits (cp.async groups only)
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
   switch (bits) {
     case 2: return launch_gemv_b<2>(X, m, n, k, packed, scales, zeros, Y, y_f32, stream);
@@ -1368,13 +1357,9 @@ cudaError_t launch_group_cfg(const GemvLayer* layers, int count, int M, bool y_f
     grp.tile_end[i] = tiles;
   }
   auto kern = gemm_gemv_group_kernel<NT, RT, S>;
-  static int attr_bytes = 0;  // per template instance: the largest size set so far
-  if (static_cast<int>(smem) > attr_bytes) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    attr_bytes = static_cast<int>(smem);
-  }
+  static SmemAttr smem_attr;  // per template instance
+  const cudaError_t ea = smem_attr.ensure(kern, static_cast<int>(smem));
+  if (ea != cudaSuccess) return ea;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(tiles), 1, 1);
   cfg.blockDim = dim3(32 * S, 1, 1);
@@ -1418,7 +1403,8 @@ cudaError_t launch_group_rt(const GemvLayer* layers, int count, int M, bool y_f3
 int gemm_gemv_group_max() { return kMaxGroup; }
 
 cudaError_t launch_gemm_gemv_group(const GemvCall* calls, int count, int64_t M, bool y_f32,
-                                   cudaStream_t stream) {
+                                   uint32_t* flags, cudaStream_t stream) {
+  (void)flags;
   if (count < 1 || count > kMaxGroup) return cudaErrorInvalidValue;
   GemvLayer layers[kMaxGroup];
   int64_t rows = 0;
@@ -1456,21 +1442,45 @@ static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 constexpr int kMaxDevices = 64;
 std::mutex g_static_mu;
 void* g_static_ptr[kMaxDevices] = {};
+void* g_static_ctx[kMaxDevices] = {};
+
+// The current context (the device's primary context under the runtime), from
+// the driver entry point looked up through the runtime.
+void* current_context() {
+  using GetCtx = int (*)(void**);
+  static GetCtx fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<GetCtx>(p);
+  });
+  void* ctx = nullptr;
+  if (fn) fn(&ctx);
+  return ctx;
+}
 
 // The device address of g_static_scratch on the current device.  In host
 // code the array's name is only a host-side stand-in, so the address is
-// looked up (once per device, with that device current) and cached.
+// looked up with that device current and cached per device, together with
+// the context it belongs to: after a cudaDeviceReset the device gets a new
+// primary context (and a new copy of the array), and the address is looked
+// up again.
 cudaError_t static_scratch(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  void* ctx = current_context();
   std::lock_guard<std::mutex> lock(g_static_mu);
-  if (!g_static_ptr[dev]) {
+  if (!g_static_ptr[dev] || g_static_ctx[dev] != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_static_scratch);
     if (e != cudaSuccess) return e;
     g_static_ptr[dev] = p;
+    g_static_ctx[dev] = ctx;
   }
   *out = g_static_ptr[dev];
   return cudaSuccess;

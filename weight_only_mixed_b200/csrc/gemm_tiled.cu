@@ -34,6 +34,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <mutex>
+
 #include "dequant.cuh"
 #include "internal.h"
 #include "ptx.cuh"
@@ -61,18 +63,16 @@ constexpr int p_stage_bytes() {
   return kBM * 16 * B;
 }
 
-// Stage counts and the shared-memory budget.  The decode tile (BN = 16) aims
-// for two CTAs per SM and spends what is left of 112 KB on packed-W stages;
-// wider tiles use one CTA per SM and up to 227 KB, so that many bytes of
-// weights are in flight either way.
+// Stage counts and the shared-memory budget: one CTA per SM, up to 227 KB,
+// what is left after the X and A stages going to packed-W stages.
 template <int B, int BN>
 struct Cfg {
-  static constexpr int kSX = BN == 16 ? 8 : (BN == 256 ? 3 : 4);
+  static constexpr int kSX = BN == 256 ? 3 : 4;
   static constexpr int kXStage = BN * 128;
   static constexpr int kAStage = kBM * 128;
   static constexpr int kFixed = 1024 /* alignment slack */ + kSX * kXStage + kSA * kAStage +
                                 kSRing * kBM * 3 + 512 /* barriers, TMEM address, flag */;
-  static constexpr int kBudget = BN == 16 ? 112 * 1024 : 227 * 1024;
+  static constexpr int kBudget = 227 * 1024;
   static constexpr int kSPRaw = (kBudget - kFixed) / p_stage_bytes<B>();
   static constexpr int kSP = kSPRaw > 8 ? 8 : (kSPRaw < 2 ? 2 : kSPRaw);
   static constexpr int kSmem = kFixed + kSP * p_stage_bytes<B>();
@@ -102,7 +102,6 @@ struct Bars {
   uint64_t* pf;  // P buffer filled (tcgen05.commit)
   uint64_t* pe;  // P buffer drained by the workers
   uint64_t* mma_done;
-  uint64_t* done;  // decode tile: MMAs of group g complete (ring of 4)
   uint32_t* tmem_base;
   volatile int* abort_flag;
 };
@@ -136,18 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       uint32_t* __restrict__ flags) {
   using C = Cfg<B, BN>;
   constexpr int kSP = C::kSP;
-  // The 8 K=16 MMAs of a group go to kChains independent accumulators (MMA k
-  // into chain k mod kChains).  With the 16-wide decode tile each MMA is tiny
-  // and a single dependent chain runs at the tensor core's latency, not its
-  // throughput; four chains overlap.  Wider tiles keep one chain.
-  constexpr int kChains = BN == 16 ? 4 : 1;
-  // Decode tile: one commit per group (done[g % 4]) stands for "A stages,
-  // X stages and P buffer of group g are free / ready"; the MMA thread waits
-  // only for the second k-block of a group, which both producers publish
-  // after the first.  This keeps the single issuing thread's per-group
-  // latency (waits, commits) small next to its eight MMAs.
-  constexpr bool kDec = BN == 16;
-  constexpr int kCols = 2 * kChains * BN;  // two P buffers of kChains accumulators
+  constexpr int kCols = 2 * BN;  // two P buffers
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -167,8 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   sh.pf = sh.p_empty + kSP;
   sh.pe = sh.pf + 2;
   sh.mma_done = sh.pe + 2;
-  sh.done = sh.mma_done + 1;
-  sh.tmem_base = reinterpret_cast<uint32_t*>(sh.done + 4);
+  sh.tmem_base = reinterpret_cast<uint32_t*>(sh.mma_done + 1);
   sh.abort_flag = reinterpret_cast<volatile int*>(sh.tmem_base + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -184,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kSX; ++i) {
-      mbar_init(&sh.x_full[i], BN == 16 ? 32 : 1);  // decode: one arrival per producer lane
+      mbar_init(&sh.x_full[i], 1);
       mbar_init(&sh.x_empty[i], 1);
     }
     for (int i = 0; i < kSA; ++i) {
@@ -200,7 +187,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sh.pe[i], kWorkers);
     }
     mbar_init(sh.mma_done, 1);
-    for (int i = 0; i < 4; ++i) mbar_init(&sh.done[i], 1);
     *sh.abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -214,51 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *sh.tmem_base;
 
-  if (warp == kWarpX && BN == 16) {
-    // ---------------- X producer, decode tile ----------------
-    // The 16 x 64 X tile of a k-block is only a few rows of activations that
-    // every CTA reads; all 32 lanes copy it with 16-byte cp.async (rows >= M
-    // zero-filled), kXAhead k-blocks ahead, and publish a stage once its
-    // copies have landed (wait_group, then a proxy fence for tcgen05.mma).
-    constexpr int kXAhead = 4;
-    static_assert(BN != 16 || kXAhead < C::kSX, "X lookahead must leave a free stage");
-    auto copy_kblock = [&](int kb) {
-      const int s = kb % C::kSX;
-      uint8_t* dst = xbuf + s * C::kXStage;
-      const int64_t k0 = static_cast<int64_t>(2 * g_begin + kb) * kBK;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int v = lane + 32 * j;  // 16 rows x 8 chunks of 16 bytes
-        const int r = v >> 3, c = v & 7;
-        const bool in = (m0 + r) < M;
-        const uint16_t* src = in ? X + static_cast<int64_t>(m0 + r) * K + k0 + 8 * c : X;
-        cp_async_16(dst + r * 128 + ((c ^ (r & 7)) << 4), src, in ? 16u : 0u);
-      }
-    };
-    bool ok = true;
-    for (int kb = 0; kb < kXAhead && kb < KB; ++kb) {
-      copy_kblock(kb);  // the first stages are free
-      cp_async_commit();
-    }
-    for (int kb = 0; kb < KB && ok; ++kb) {
-      const int kn = kb + kXAhead;
-      if (kn < KB) {
-        bool w = true;
-        if (kn >= C::kSX) {  // the stage held k-block kn - kSX: its group's MMAs must be done
-          const int gx = (kn - C::kSX) >> 1;
-          w = wait_or_abort(&sh.done[gx & 3], (gx >> 2) & 1, sh, flags);
-        }
-        ok = __all_sync(0xffffffffu, w);
-        if (ok) copy_kblock(kn);
-      }
-      cp_async_commit();  // possibly empty: keeps one group per k-block
-      cp_async_wait<kXAhead>();  // the group of k-block kb has landed
-      fence_proxy_async_smem();
-      mbar_arrive(&sh.x_full[kb % C::kSX]);
-    }
-    cp_async_wait<0>();  // nothing in flight past this point
-    __syncwarp();
-  } else if (warp == kWarpX) {
+  if (warp == kWarpX) {
     // ---------------- X producer (TMA) ----------------
     if (lane == 0) {
       prefetch_tmap(&tmap_x);
@@ -339,28 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = wait_or_abort(&sh.pe[buf], ((g >> 1) & 1) ^ 1, sh, flags);
         if (!ok) break;
         tc_fence_after_sync();
-        const uint32_t d = tmem + static_cast<uint32_t>(buf * kChains * BN);
-        if constexpr (kDec) {
-          const int kb1 = 2 * g + 1;
-          ok = wait_or_abort(&sh.a_full[kb1 % kSA], (kb1 / kSA) & 1, sh, flags) &&
-               wait_or_abort(&sh.x_full[kb1 % C::kSX], (kb1 / C::kSX) & 1, sh, flags);
-          if (!ok) break;
-          tc_fence_after_sync();
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int kb = 2 * g + h;
-            const uint64_t da = sw128_desc(smem_u32(abuf + (kb % kSA) * C::kAStage));
-            const uint64_t db = sw128_desc(smem_u32(xbuf + (kb % C::kSX) * C::kXStage));
-#pragma unroll
-            for (int k = 0; k < kBK / 16; ++k) {
-              const int kk = h * (kBK / 16) + k;
-              umma_bf16_ss(d + static_cast<uint32_t>((kk % kChains) * BN), da + 2 * k, db + 2 * k,
-                           idesc, kk >= kChains ? 1u : 0u);
-            }
-          }
-          umma_commit(&sh.done[g & 3]);
-          continue;
-        }
+        const uint32_t d = tmem + static_cast<uint32_t>(buf * BN);
 #pragma unroll 1
         for (int h = 0; h < 2 && ok; ++h) {
           const int kb = 2 * g + h;
@@ -374,8 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k) {  // +32 bytes along K per MMA: +2 in the address field
             const int kk = h * (kBK / 16) + k;  // MMA index within the group
-            umma_bf16_ss(d + static_cast<uint32_t>((kk % kChains) * BN), da + 2 * k, db + 2 * k,
-                         idesc, kk >= kChains ? 1u : 0u);
+            umma_bf16_ss(d, da + 2 * k, db + 2 * k, idesc, kk > 0 ? 1u : 0u);
           }
           umma_commit(&sh.a_empty[sa]);
           umma_commit(&sh.x_empty[sx]);
@@ -402,14 +322,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (g < ng) {
         // ---- dequantize group g into A stages 2g, 2g+1 ----
         const int sp = g % kSP;
-        if constexpr (kDec) {  // A stages of group g - 2 are free once its MMAs are done
-          ok = (g < 2 || wait_or_abort(&sh.done[(g - 2) & 3], ((g - 2) >> 2) & 1, sh, flags)) &&
-               wait_or_abort(&sh.p_full[sp], (g / kSP) & 1, sh, flags);
-        } else {
-          ok = wait_or_abort(&sh.a_empty[(2 * g) % kSA], (((2 * g) / kSA) & 1) ^ 1, sh, flags) &&
-               wait_or_abort(&sh.a_empty[(2 * g + 1) % kSA], (((2 * g + 1) / kSA) & 1) ^ 1, sh, flags) &&
-               wait_or_abort(&sh.p_full[sp], (g / kSP) & 1, sh, flags);
-        }
+        ok = wait_or_abort(&sh.a_empty[(2 * g) % kSA], (((2 * g) / kSA) & 1) ^ 1, sh, flags) &&
+             wait_or_abort(&sh.a_empty[(2 * g + 1) % kSA], (((2 * g + 1) / kSA) & 1) ^ 1, sh, flags) &&
+             wait_or_abort(&sh.p_full[sp], (g / kSP) & 1, sh, flags);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         const uint8_t* pst = pbuf + sp * p_stage_bytes<B>();
@@ -442,17 +357,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---- fold P_{g-1} into the accumulators: acc += s[n, g-1] * P ----
         const int j = g - 1;
         const int buf = j & 1;
-        if constexpr (kDec)
-          ok = __all_sync(0xffffffffu, wait_or_abort(&sh.done[j & 3], (j >> 2) & 1, sh, flags));
-        else
-          ok = __all_sync(0xffffffffu, wait_or_abort(&sh.pf[buf], (j >> 1) & 1, sh, flags));
+        ok = __all_sync(0xffffffffu, wait_or_abort(&sh.pf[buf], (j >> 1) & 1, sh, flags));
         if (!ok) break;
         tc_fence_after_sync();
         const float s =
             __half2float(__ushort_as_half(sring[(j % kSRing) * kBM + 32 * q + lane]));
         const uint32_t base = tmem + (static_cast<uint32_t>(32 * q) << 16) +
-                              static_cast<uint32_t>(buf * kChains * BN + hcol * kHalf);
-        if constexpr (kHalf % 16 == 0) {
+                              static_cast<uint32_t>(buf * BN + hcol * kHalf);
+        static_assert(kHalf % 16 == 0, "column halves are whole 16-column blocks");
+        {
           // Four column blocks of 16 per TMEM wait (the wait covers every
           // load issued before it): one wait per block left the fold
           // latency-bound, about 10 % of the kernel's time at M >= 1024.
@@ -468,19 +381,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int i = 0; i < 16; ++i)
                 acc[16 * (c + e) + i] = fmaf(s, __uint_as_float(r[e][i]), acc[16 * (c + e) + i]);
-          }
-        } else {
-          // Decode tile: sum the kChains partial accumulators in a fixed order.
-          uint32_t r[kChains][8];
-#pragma unroll
-          for (int c = 0; c < kChains; ++c) tmem_ld_32x32b_x8(base + static_cast<uint32_t>(c * BN), r[c]);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float v = __uint_as_float(r[0][i]);
-#pragma unroll
-            for (int c = 1; c < kChains; ++c) v += __uint_as_float(r[c][i]);
-            acc[i] = fmaf(s, v, acc[i]);
           }
         }
         tc_fence_before_sync();
@@ -566,18 +466,11 @@ cudaError_t launch_cfg(const uint16_t* X, int M, int N, int K, const uint32_t* p
                             static_cast<uint64_t>(K) * B / 32, static_cast<uint64_t>(N),
                             static_cast<uint64_t>(K) * B / 8, 4 * B, kBM, swz))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(gemm_tiled_kernel<B, BN>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  static SmemAttr smem_attr;  // per template instance
+  const cudaError_t e = smem_attr.ensure(gemm_tiled_kernel<B, BN>, C::kSmem);
   if (e != cudaSuccess) return e;
-  // Ask for the largest shared-memory carveout so that two decode CTAs fit
-  // on an SM (the default carveout may hold only one).
-  e = cudaFuncSetAttribute(gemm_tiled_kernel<B, BN>,
-                           cudaFuncAttributePreferredSharedMemoryCarveout,
-                           static_cast<int>(cudaSharedmemCarveoutMaxShared));
-  if (e != cudaSuccess) return e;
-  int sms = 148, dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
   const int G = K / kGroup;
   const int row_blocks = (N + kBM - 1) / kBM;
   const int col_blocks = (M + BN - 1) / BN;
@@ -598,19 +491,35 @@ cudaError_t launch_cfg(const uint16_t* X, int M, int N, int K, const uint32_t* p
   // cluster placement, not only shared memory, limits residency.
   int C_split = 1;
   if (BN <= 64) {
-    static int max_active[kMaxCluster + 1] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};
+    // Resident clusters per cluster size, per device (the query depends on
+    // the device's SMs); filled on first use under a lock, since calls may
+    // come from several host threads.
+    constexpr int kDevs = 64;
+    static std::mutex mu;
+    static int max_active[kDevs][kMaxCluster + 1];
+    static bool known[kDevs][kMaxCluster + 1];
     const int tiles = row_blocks * col_blocks;
     for (int c = kMaxCluster; c >= 2; --c) {
       if (c > G / 4) continue;
-      if (max_active[c] < 0) {
-        attr[0].val.clusterDim.z = static_cast<unsigned>(c);
-        cfg.gridDim = dim3(1, 1, static_cast<unsigned>(c));
-        int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, gemm_tiled_kernel<B, BN>, &cfg) != cudaSuccess) n = 0;
-        cudaGetLastError();
-        max_active[c] = n;
+      int active = 0;
+      {
+        std::lock_guard<std::mutex> lock(mu);
+        if (dev < 0 || dev >= kDevs || !known[dev][c]) {
+          attr[0].val.clusterDim.z = static_cast<unsigned>(c);
+          cfg.gridDim = dim3(1, 1, static_cast<unsigned>(c));
+          int n = 0;
+          if (cudaOccupancyMaxActiveClusters(&n, gemm_tiled_kernel<B, BN>, &cfg) != cudaSuccess) n = 0;
+          cudaGetLastError();
+          if (dev >= 0 && dev < kDevs) {
+            max_active[dev][c] = n;
+            known[dev][c] = true;
+          }
+          active = n;
+        } else {
+          active = max_active[dev][c];
+        }
       }
-      if (tiles <= max_active[c]) {
+      if (tiles <= active) {
         C_split = c;
         break;
       }
@@ -626,13 +535,12 @@ cudaError_t launch_cfg(const uint16_t* X, int M, int N, int K, const uint32_t* p
                             y_f32 ? 1 : 0, per_slice, flags);
 }
 
-// Tile width: BN = 16 for decode batches (M <= 16), otherwise the smallest of
-// 64 / 128 / 256 that covers M, so padding rows cost no more than needed.
+// Tile width: the smallest of 64 / 128 / 256 that covers M, so padding rows
+// cost no more than needed.
 template <int B>
 cudaError_t launch_b(const uint16_t* X, int M, int N, int K, const uint32_t* packed,
                      const uint16_t* scales, const uint8_t* zeros, void* Y, bool y_f32,
-                     bool decode, uint32_t* flags, cudaStream_t stream) {
-  if (decode) return launch_cfg<B, 16>(X, M, N, K, packed, scales, zeros, Y, y_f32, flags, stream);
+                     uint32_t* flags, cudaStream_t stream) {
   if (M <= 64) return launch_cfg<B, 64>(X, M, N, K, packed, scales, zeros, Y, y_f32, flags, stream);
   if (M <= 128) return launch_cfg<B, 128>(X, M, N, K, packed, scales, zeros, Y, y_f32, flags, stream);
   return launch_cfg<B, 256>(X, M, N, K, packed, scales, zeros, Y, y_f32, flags, stream);
@@ -642,17 +550,16 @@ cudaError_t launch_b(const uint16_t* X, int M, int N, int K, const uint32_t* pac
 
 cudaError_t launch_gemm_tiled(const uint16_t* X, int64_t M, int64_t N, int64_t K, int bits,
                               const uint32_t* packed, const uint16_t* scales, const uint8_t* zeros,
-                              void* Y, bool y_f32, bool decode, uint32_t* flags,
-                              cudaStream_t stream) {
+                              void* Y, bool y_f32, uint32_t* flags, cudaStream_t stream) {
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
   switch (bits) {
-    case 2: return launch_b<2>(X, m, n, k, packed, scales, zeros, Y, y_f32, decode, flags, stream);
-    case 3: return launch_b<3>(X, m, n, k, packed, scales, zeros, Y, y_f32, decode, flags, stream);
-    case 4: return launch_b<4>(X, m, n, k, packed, scales, zeros, Y, y_f32, decode, flags, stream);
-    case 5: return launch_b<5>(X, m, n, k, packed, scales, zeros, Y, y_f32, decode, flags, stream);
-    case 6: return launch_b<6>(X, m, n, k, packed, scales, zeros, Y, y_f32, decode, flags, stream);
-    case 7: return launch_b<7>(X, m, n, k, packed, scales, zeros, Y, y_f32, decode, flags, stream);
-    case 8: return launch_b<8>(X, m, n, k, packed, scales, zeros, Y, y_f32, decode, flags, stream);
+    case 2: return launch_b<2>(X, m, n, k, packed, scales, zeros, Y, y_f32, flags, stream);
+    case 3: return launch_b<3>(X, m, n, k, packed, scales, zeros, Y, y_f32, flags, stream);
+    case 4: return launch_b<4>(X, m, n, k, packed, scales, zeros, Y, y_f32, flags, stream);
+    case 5: return launch_b<5>(X, m, n, k, packed, scales, zeros, Y, y_f32, flags, stream);
+    case 6: return launch_b<6>(X, m, n, k, packed, scales, zeros, Y, y_f32, flags, stream);
+    case 7: return launch_b<7>(X, m, n, k, packed, scales, zeros, Y, y_f32, flags, stream);
+    case 8: return launch_b<8>(X, m, n, k, packed, scales, zeros, Y, y_f32, flags, stream);
     default: return cudaErrorInvalidValue;
   }
 }

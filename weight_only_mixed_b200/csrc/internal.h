@@ -6,9 +6,32 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 namespace slq {
 
 constexpr int kGroup = 128;  // group size along K fixed by the format
+
+// The dynamic shared-memory limit set on one kernel, per device (a function
+// attribute belongs to the device's context).  One static instance per
+// kernel; safe when launches come from several host threads.
+struct SmemAttr {
+  std::mutex mu;
+  int bytes[64] = {};
+  template <typename F>
+  cudaError_t ensure(F kernel, int n) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= 0 && dev < 64 && bytes[dev] >= n) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, n);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               static_cast<int>(cudaSharedmemCarveoutMaxShared));
+    if (e == cudaSuccess && dev >= 0 && dev < 64) bytes[dev] = n;
+    return e;
+  }
+};
 
 // Flag bits (same values as SLQ_FLAG_* in slq.h).
 constexpr uint32_t kFlagNonfinite = 1u;
@@ -38,11 +61,11 @@ cudaError_t launch_gemm_decode(const uint16_t* X, int64_t M, int64_t N, int64_t 
 // device (0 when no row tile is split).
 size_t gemm_decode_workspace_bytes(int64_t N, int64_t K, int bits);
 
-// Split-K GEMV for M <= 16 with no workspace: a CTA per 16-row tile, its
-// warps split K, partial tiles added in shared memory.
+// Split-K GEMV for M <= 16 with no workspace: a CTA per 16- or 32-row tile,
+// its warps split K, partial tiles added in shared memory.
 cudaError_t launch_gemm_gemv(const uint16_t* X, int64_t M, int64_t N, int64_t K, int bits,
                              const uint32_t* packed, const uint16_t* scales, const uint8_t* zeros,
-                             void* Y, bool y_f32, cudaStream_t stream);
+                             void* Y, bool y_f32, uint32_t* flags, cudaStream_t stream);
 
 // One layer of a grouped GEMV launch.
 struct GemvCall {
@@ -59,7 +82,7 @@ struct GemvCall {
 // launch of the split-K GEMV kernel.
 int gemm_gemv_group_max();
 cudaError_t launch_gemm_gemv_group(const GemvCall* calls, int count, int64_t M, bool y_f32,
-                                   cudaStream_t stream);
+                                   uint32_t* flags, cudaStream_t stream);
 
 // Largest N the decode kernel accepts (the fixed tile-counter region).
 int64_t gemm_decode_max_n();
@@ -74,12 +97,12 @@ cudaError_t launch_gemm_decode_static(const uint16_t* X, int64_t M, int64_t N, i
                                       cudaStream_t stream);
 
 // Dequantize-GEMM on tcgen05 (TMA + dequant to shared memory + tcgen05.mma
-// with TMEM accumulators).  decode = true selects the 16-wide activation tile
-// with split-K over a cluster (M <= 16); otherwise the tile width follows M.
+// with TMEM accumulators); the tile width follows M, and K is split over a
+// thread-block cluster for narrow tiles.
 cudaError_t launch_gemm_tiled(const uint16_t* X, int64_t M, int64_t N, int64_t K, int bits,
                               const uint32_t* packed, const uint16_t* scales,
-                              const uint8_t* zeros, void* Y, bool y_f32, bool decode,
-                              uint32_t* flags, cudaStream_t stream);
+                              const uint8_t* zeros, void* Y, bool y_f32, uint32_t* flags,
+                              cudaStream_t stream);
 
 cudaError_t launch_ear_kl(const uint16_t* a, const uint16_t* b, int64_t T, int64_t V,
                           float temperature, float* ear_tok, float* kl_tok,

@@ -187,19 +187,18 @@ slq_status slq_gemm_ex(const void* X_bf16, int64_t M, int64_t N, int64_t K, int 
   const uint16_t* X = static_cast<const uint16_t*>(X_bf16);
   const uint16_t* sc = static_cast<const uint16_t*>(scales_f16);
   if (path == SLQ_GEMM_GEMV)
-    return from_cuda(slq::launch_gemm_gemv(X, M, N, K, bits, packed, sc, zeros, Y, f32, s));
+    return from_cuda(slq::launch_gemm_gemv(X, M, N, K, bits, packed, sc, zeros, Y, f32, flags, s));
   if (path == SLQ_GEMM_DECODE)
     return from_cuda(
         slq::launch_gemm_decode(X, M, N, K, bits, packed, sc, zeros, Y, f32, workspace, flags, s));
-  return from_cuda(slq::launch_gemm_tiled(X, M, N, K, bits, packed, sc, zeros, Y, f32, false, flags, s));
+  return from_cuda(slq::launch_gemm_tiled(X, M, N, K, bits, packed, sc, zeros, Y, f32, flags, s));
 }
 
 slq_status slq_gemm(const void* X_bf16, int64_t M, int64_t N, int64_t K, int bits,
                     const uint32_t* packed, const void* scales_f16, const uint8_t* zeros, void* Y,
-                    slq_dtype y_dtype, void* workspace, size_t workspace_bytes, uint32_t* flags,
-                    void* stream) {
+                    slq_dtype y_dtype, uint32_t* flags, void* stream) {
   return slq_gemm_ex(X_bf16, M, N, K, bits, packed, scales_f16, zeros, Y, y_dtype, SLQ_GEMM_AUTO,
-                     workspace, workspace_bytes, flags, stream);
+                     nullptr, 0, flags, stream);
 }
 
 int slq_gemm_group_max(void) { return slq::gemm_gemv_group_max(); }
@@ -236,7 +235,7 @@ slq_status slq_gemm_group(const slq_gemm_layer* layers, int count, int64_t M, sl
   }
   const slq_status dev = check_device();
   if (dev != SLQ_OK) return dev;
-  return from_cuda(slq::launch_gemm_gemv_group(calls, n, M, y_dtype == SLQ_DTYPE_F32,
+  return from_cuda(slq::launch_gemm_gemv_group(calls, n, M, y_dtype == SLQ_DTYPE_F32, flags,
                                                static_cast<cudaStream_t>(stream)));
 }
 
