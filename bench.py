@@ -30,6 +30,7 @@ ncu captures use.  SPEC is one of
   ear:T:V:tau               one EAR/KL reduction
   eartopk:T:V:tau:K         one top-K EAR/KL reduction
   quantize:N:K:b            one quantize+pack
+  gridnoise:N:K:b           one grid-noise pass (gamma, asymmetric and symmetric SSE)
 
 --impl reference times the CPU oracle (the plain reference implementation
 of the same arithmetic) on a bounded sample of the same workload, on the
@@ -532,7 +533,23 @@ def other_rows(args, slq, synth, torch, dev, stream, hbm_peak, tc_peak, rank):
     rows["quantize_block"] = {"GBps": round(qbytes / (ms * 1e-3) / 1e9, 1),
                               "frac_hbm": round(qbytes / (ms * 1e-3) / 1e9 / hbm_peak, 3),
                               "us": round(ms * 1e3, 2), "bytes": qbytes}
-    del Ws, outs
+    # Grid noise (gamma, asymmetric and symmetric SSE) of the same 7 weights.
+    gouts = [[torch.empty((N, K // 128), dtype=torch.float32, device=dev) for _ in range(3)]
+             for (_, N, K, b) in QWEN3_8B_BLOCK]
+    L = slq.lib()
+
+    def gstep():
+        for W, o, (_, N, K, b) in zip(Ws, gouts, QWEN3_8B_BLOCK):
+            rc = L.slq_grid_noise(W.data_ptr(), N, K, b, o[0].data_ptr(), o[1].data_ptr(),
+                                  o[2].data_ptr(), None, stream.cuda_stream)
+            assert rc == 0
+
+    ms = time_ms(torch, stream, gstep, 10)
+    gbytes = sum(N * K * 2 + 12 * N * (K // 128) for _, N, K, b in QWEN3_8B_BLOCK)
+    rows["grid_noise_block"] = {"GBps": round(gbytes / (ms * 1e-3) / 1e9, 1),
+                                "frac_hbm": round(gbytes / (ms * 1e-3) / 1e9 / hbm_peak, 3),
+                                "us": round(ms * 1e3, 2), "bytes": gbytes}
+    del Ws, outs, gouts
 
     # Decode sweep N = K = 8192 at every b, M in {1, 16}.
     sweep = {}
@@ -928,6 +945,13 @@ def run_case(args):
 
         def fn():
             slq.quantize(W, b, out=q, stream=stream)
+        per_call = 1
+    elif kind == "gridnoise":
+        N, K, b = vals
+        W = synth.weights_torch(N, K, device=dev)
+
+        def fn():
+            slq.grid_noise(W, b, stream=stream)
         per_call = 1
     else:
         raise SystemExit(f"unknown --case {args.case}")

@@ -307,6 +307,39 @@ slq_status slq_ear_kl_topk(const void *logits_p_bf16, const void *logits_q_bf16,
 /* Largest top_k slq_ear_kl_topk takes (16). */
 int slq_ear_kl_topk_max(void);
 
+/*
+ * slq_grid_noise -- per-group rounding noise of the asymmetric b-bit grid
+ * (the format's) and of the symmetric one it replaces.
+ *
+ * Source: wispaper.ai blog, the section on the gamma^2 variance law, and the
+ * gist.science summary, Methodology section 1 "Theoretical Foundation": for a
+ * group with range R = max w - min w and largest magnitude M = max |w|,
+ * gamma = 2 M / R; a symmetric grid over [-M, M] has gamma times the step of
+ * an asymmetric grid over [min w, max w], so gamma^2 times its rounding-noise
+ * variance.  For every 128-weight group g (row n, groups along K) this call
+ * writes, with L = 2^bits - 1:
+ *   gamma[g]    = 2 M / R, or 1 when R = 0
+ *   sse_asym[g] = sum over the group of (w - nearest point of
+ *                 {min w + i R / L : i = 0..L})^2
+ *   sse_sym[g]  = the same for {-M + i 2 M / L : i = 0..L}
+ * The grids are continuous (no fp16 scale or integer zero point): this is the
+ * quantity the pages' variance argument speaks of, not the stored format's
+ * error.  Group statistics are exact; per-weight errors are binary32.
+ *
+ * W_bf16     [N, K] row-major bf16, device, 16-byte aligned.
+ * N, K       N >= 0 (0 launches nothing), K a positive multiple of 128.
+ * bits       2..8.
+ * gamma, sse_asym, sse_sym  [N, K / 128] fp32, device, written; disjoint
+ *            from W.
+ * flags      device uint32 or NULL: SLQ_FLAG_NONFINITE when a group holds a
+ *            NaN or an infinity (that group's outputs are then meaningless).
+ * Errors: SLQ_ERR_INVALID_ARGUMENT for sizes, bits, alignment or overlap
+ * before any launch; SLQ_ERR_CUDA for a failed launch.
+ */
+slq_status slq_grid_noise(const void *W_bf16, int64_t N, int64_t K, int bits,
+                          float *gamma, float *sse_asym, float *sse_sym,
+                          uint32_t *flags, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -210,3 +210,18 @@ def test_ear_kl_topk_validation():
         assert call(**bad) == slq.SLQ_ERR_INVALID_ARGUMENT, bad
     assert call(T=0) == slq.SLQ_OK
     assert call() in (slq.SLQ_OK, slq.SLQ_ERR_UNSUPPORTED_DEVICE)
+
+
+def test_grid_noise_validation():
+    def call(W=FAKE, N=4, K=256, bits=4, g=FAKE + (1 << 24), a=FAKE + (2 << 24), s=FAKE + (3 << 24),
+             flags=None):
+        return L.slq_grid_noise(W, N, K, bits, g, a, s, flags, None)
+
+    for bad in [dict(N=-1), dict(K=0), dict(K=200), dict(bits=1), dict(bits=9), dict(W=None),
+                dict(g=None), dict(a=None), dict(s=None), dict(W=FAKE + 8), dict(g=FAKE + (1 << 24) + 2),
+                dict(flags=FAKE + (4 << 24) + 1),
+                dict(g=FAKE + 1024),                # output overlaps W
+                dict(N=1 << 31)]:
+        assert call(**bad) == slq.SLQ_ERR_INVALID_ARGUMENT, bad
+    assert call(N=0) == slq.SLQ_OK
+    assert call() in (slq.SLQ_OK, slq.SLQ_ERR_UNSUPPORTED_DEVICE)

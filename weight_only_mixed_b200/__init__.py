@@ -95,6 +95,8 @@ _lib.slq_ear_kl_topk.argtypes = [_P, _P, _I64, _I64, _I, ctypes.c_float, _P, _P,
 _lib.slq_ear_kl_topk.restype = _I
 _lib.slq_ear_kl_topk_max.argtypes = []
 _lib.slq_ear_kl_topk_max.restype = _I
+_lib.slq_grid_noise.argtypes = [_P, _I64, _I64, _I, _P, _P, _P, _P, _P]
+_lib.slq_grid_noise.restype = _I
 
 
 def lib() -> ctypes.CDLL:
@@ -456,3 +458,21 @@ def ear_kl(a, b, temperature: float = 1.0, means: bool = True, flags=None, strea
                                    _ptr(em), _ptr(km), _ptr(flags), _stream_ptr(stream, dev)),
                    "slq_ear_kl")
     return ear, kl, em, km
+
+
+def grid_noise(W, bits: int, flags=None, stream=None):
+    """Per 128-weight group of a [N, K] bf16 CUDA tensor: gamma = 2 max|w| /
+    (max w - min w) and the rounding SSE of the asymmetric and the symmetric
+    continuous b-bit grids (slq_grid_noise).  Returns (gamma, sse_asym,
+    sse_sym), fp32 [N, K/128] each."""
+    import torch
+    _require(W, "W", (torch.bfloat16,), ndim=2)
+    N, K = W.shape
+    _require_bits_k(bits, K)
+    _require_flags(flags)
+    dev = _require_cuda(W=W, flags=flags)
+    with _on(dev):
+        outs = [torch.empty((N, K // GROUP), dtype=torch.float32, device=dev) for _ in range(3)]
+        _check(_lib.slq_grid_noise(_ptr(W), N, K, bits, _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]),
+                                   _ptr(flags), _stream_ptr(stream, dev)), "slq_grid_noise")
+    return tuple(outs)

@@ -77,44 +77,6 @@ __device__ __forceinline__ void push(RowStat& st, float a, float b, float c) {
   st.b.s += ex2((b - st.b.m) * c);
 }
 
-// ---------------------------------------------------------------------------
-// Packed binary32 pairs (sm_100 f32x2 instructions: one issue, two lanes).
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint64_t pk(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ float pk_lo(uint64_t v) {
-  float lo, hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  return lo;
-}
-__device__ __forceinline__ float pk_hi(uint64_t v) {
-  float lo, hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  return hi;
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
 // The two bf16 logits of one 32-bit word as a packed binary32 pair (exact).
 __device__ __forceinline__ uint64_t bf16x2_f32x2(uint32_t w) { return pk(bf16_lo(w), bf16_hi(w)); }
 __device__ __forceinline__ uint64_t ex2x2(uint64_t x) { return pk(ex2(pk_lo(x)), ex2(pk_hi(x))); }

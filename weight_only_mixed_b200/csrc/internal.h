@@ -115,4 +115,9 @@ cudaError_t launch_ear_kl_topk(const uint16_t* a, const uint16_t* b, int64_t T, 
                                float temperature, float* ear_tok, float* kl_tok, double* ear_mean,
                                double* kl_mean, cudaStream_t stream);
 
+// Per-group gamma and the rounding SSE of the asymmetric and symmetric
+// continuous b-bit grids; outputs [N, K / 128] fp32.
+cudaError_t launch_grid_noise(const uint16_t* W, int64_t N, int64_t K, int bits, float* gamma,
+                              float* sse_asym, float* sse_sym, uint32_t* flags, cudaStream_t stream);
+
 }  // namespace slq

@@ -35,19 +35,6 @@ constexpr int kUnroll = 4;  // groups per warp per iteration (loads in flight)
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
-// Warp-wide float min / max in one instruction (sm_100a redux.sync); a NaN
-// input is ignored, as with fminf / fmaxf.
-__device__ __forceinline__ float warp_min(float v) {
-  float r;
-  asm volatile("redux.sync.min.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
-  return r;
-}
-__device__ __forceinline__ float warp_max(float v) {
-  float r;
-  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
-  return r;
-}
-
 // rne(fl32(w / s)) for the encode.  With r = RN(1/s), t = RN(w r) differs from
 // the IEEE quotient fl32(w / s) by at most 1.5 * 2^-23 * |t| (< 1.9e-4 for
 // |t| < 1024), so the two round to the same integer unless t lies within that

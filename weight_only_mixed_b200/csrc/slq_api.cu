@@ -323,4 +323,25 @@ slq_status slq_ear_kl(const void* logits_p_bf16, const void* logits_q_bf16, int6
       V, temperature, ear_tok, kl_tok, ear_mean, kl_mean, flags, static_cast<cudaStream_t>(stream)));
 }
 
+slq_status slq_grid_noise(const void* W_bf16, int64_t N, int64_t K, int bits, float* gamma,
+                          float* sse_asym, float* sse_sym, uint32_t* flags, void* stream) {
+  if (N < 0 || N > kMaxDim || !valid_k(K) || !valid_bits(bits) || !product_ok(N, K))
+    return SLQ_ERR_INVALID_ARGUMENT;
+  if (N == 0) return SLQ_OK;
+  if (!W_bf16 || !gamma || !sse_asym || !sse_sym) return SLQ_ERR_INVALID_ARGUMENT;
+  if (!aligned(W_bf16, 16) || !aligned(gamma, 4) || !aligned(sse_asym, 4) || !aligned(sse_sym, 4) ||
+      (flags && !aligned(flags, 4)))
+    return SLQ_ERR_INVALID_ARGUMENT;
+  const int64_t G = N * (K / slq::kGroup);
+  const Range ins[1] = {range_of(W_bf16, N * K * 2)};
+  const Range outs[4] = {range_of(gamma, G * 4), range_of(sse_asym, G * 4), range_of(sse_sym, G * 4),
+                         range_of(flags, flags ? 4 : 0)};
+  if (!disjoint(outs, 4, ins, 1)) return SLQ_ERR_INVALID_ARGUMENT;
+  const slq_status dev = check_device();
+  if (dev != SLQ_OK) return dev;
+  return from_cuda(slq::launch_grid_noise(static_cast<const uint16_t*>(W_bf16), N, K, bits, gamma,
+                                          sse_asym, sse_sym, flags,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"
