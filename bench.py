@@ -21,8 +21,8 @@ pages' models (no checkpoints or datasets here).
   python bench.py --case SPEC [--steps K] [--warmup W]
 
 --case runs one kernel of the path on its own (W untimed launches, then K
-timed ones) and prints {"case", "avg_us", ...}: the command the profiles'
-ncu captures use.  SPEC is one of
+timed ones; with --graph the K calls replay as one CUDA graph) and prints
+{"case", "avg_us", ...}: the command the profiles' ncu captures use.  SPEC is one of
   block                     the 12 decode launches of one Qwen3-8B block step
   gemv:N:K:b:M              one dequant-GEMM on the split-K GEMV kernel (M <= 16)
   decode:N:K:b:M            one dequant-GEMM on the stream-K decode kernel (M <= 16)
@@ -917,12 +917,18 @@ def run_case(args):
         per_call = len(calls)
     elif kind in ("gemv", "decode", "tiled"):
         N, K, b, M = vals
-        qw = slq.quantize(synth.weights_torch(N, K, device=dev), b)
+        # Enough weight copies that consecutive calls miss in L2 (256 MB total).
+        W0 = synth.weights_torch(N, K, device=dev)
+        nrot = max(1, -(-(256 << 20) // weight_bytes(N, K, b)))
+        qws = [slq.quantize(W0, b)] + [slq.quantize(W0 * (1.0 + 2.0**-7 * r), b) for r in range(1, nrot)]
+        del W0
         x = synth.activations_torch(M, K, device=dev)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        it = [0]
 
         def fn():
-            slq.gemm(x, qw, out=y, path=kind, stream=stream)
+            slq.gemm(x, qws[it[0] % nrot], out=y, path=kind, stream=stream)
+            it[0] += 1
         per_call = 1
     elif kind == "ear":
         T, V, tau = vals
@@ -958,16 +964,30 @@ def run_case(args):
     for _ in range(args.warmup):
         fn()
     torch.cuda.synchronize()
+    run = fn
+    if args.graph:
+        # The calls captured in one CUDA graph: device time without the
+        # host's per-call cost (small layers take less than a Python call).
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for _ in range(args.steps):
+                fn()
+        graph.replay()
+        torch.cuda.synchronize()
+        run = graph.replay
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
-        fn()
+    if args.graph:
+        run()
+    else:
+        for _ in range(args.steps):
+            run()
     e1.record(stream)
     e1.synchronize()
     us = e0.elapsed_time(e1) * 1e3 / max(1, args.steps)
     print(json.dumps({"case": args.case, "avg_us_per_call": round(us, 3), "launches_per_call": per_call,
-                      "calls": args.steps, "warmup": args.warmup}), flush=True)
+                      "calls": args.steps, "warmup": args.warmup, "graph": bool(args.graph)}), flush=True)
 
 
 def main():
@@ -983,6 +1003,7 @@ def main():
                     help="output rows of each projection in the oracle's GEMM sample")
     ap.add_argument("--cpu-single", action="store_true", help="cpu_baseline on one core only")
     ap.add_argument("--case", default=None, help="run one kernel on its own (see the module docstring)")
+    ap.add_argument("--graph", action="store_true", help="--case: time the calls as one captured CUDA graph")
     args = ap.parse_args()
     if args.case:
         run_case(args)

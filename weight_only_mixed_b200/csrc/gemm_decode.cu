@@ -670,14 +670,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 // through L1; the S partial tiles are added in shared memory in warp order
 // (deterministic, no cross-CTA step).
 //
-// For b <= 7 the zero point leaves the inner loop: the A pairs are the exact
-// bf16 values 128 + q (q < 128), one more mma per k-step with an all-ones A
-// gives sum_k x over the group, and the group's product is
-// s * (sum (128 + q) x - (128 + z) sum x).  For b = 2 and 4 a pair takes two
-// codes 16 bits apart in one word (one shift, one mask/or) and the
-// activation pairs are permuted to the same k order; b = 3, 5, 6, 7 take
-// consecutive codes.  For b = 8 (q up to 255 is not 128 + q in bf16) the
-// pairs are (q - z) as above.
+// The zero point leaves the inner loop: the A pairs are the codes themselves
+// as exact bf16 values code * 2^(c - 133) (pair_sub), the activation pairs
+// that meet them are x * 2^(E - c) for one exponent E per group, one more mma
+// per k-step with A = 2^(c - 133) gives Sx = sum_k x 2^(E - 133), and the
+// group's product is s * 2^(133 - E) * (sum q x 2^(E - 133) - z Sx), every
+// scaling a power of two.  For b = 2 and 4 a pair takes two codes 16 bits
+// apart in one word (one mask; one shift by 8 per word for the codes in the
+// upper bytes) and the activation pairs are permuted to the same k order.
 // ---------------------------------------------------------------------------
 template <int B>
 __device__ __forceinline__ void lds_unit(const uint8_t* p, uint32_t (&w)[B]) {
@@ -697,40 +697,6 @@ __device__ __forceinline__ void lds_unit(const uint8_t* p, uint32_t (&w)[B]) {
 #pragma unroll
     for (int i = 0; i < B; ++i) w[i] = reinterpret_cast<const uint32_t*>(p)[i];
   }
-}
-
-// Pair p of a unit as exact bf16 (128 + q_2p, 128 + q_2p+1), b <= 7.
-template <int B>
-__device__ __forceinline__ uint32_t pair_raw(const uint32_t (&w)[B], int p) {
-  if constexpr (B == 4) {
-    const uint32_t y = __byte_perm(w[p >> 2], 0u, 0x4440 | (p & 3)) * 0x1001u;
-    return (y & 0x000F000Fu) | 0x43004300u;
-  } else if constexpr (B == 2) {
-    const uint32_t y = __byte_perm(w[p >> 3], 0u, 0x4440 | ((p >> 1) & 3)) * 0x4001u;
-    return ((y >> (4 * (p & 1))) & 0x00030003u) | 0x43004300u;
-  } else if constexpr (B == 3 || B == 5) {
-    // The pair's 2b bits t; t * (1 + 2^(16-b)) places the second code at bit
-    // 16 (3b < 17, so the two copies of t do not overlap and the sum is an or).
-    const int bit = 2 * B * p, wi = bit >> 5, sh = bit & 31;
-    const uint32_t x = sh + 2 * B <= 32 ? (w[wi] >> sh) : __funnelshift_r(w[wi], w[wi + 1], sh);
-    const uint32_t t = x & ((1u << (2 * B)) - 1u);
-    constexpr uint32_t mask = ((1u << B) - 1u) * 0x00010001u;
-    return ((t * (1u + (1u << (16 - B)))) & mask) | 0x43004300u;
-  } else {
-    return dq::code_at<B>(w, 2 * p) | (dq::code_at<B>(w, 2 * p + 1) << 16) | 0x43004300u;
-  }
-}
-
-// b = 4 and b = 2: pair p of a unit with its two codes 16 bits apart in one
-// word, as exact bf16 (128 + q, 128 + q'): one shift and one mask/or.  For
-// b = 4, pair p = 4 i + s of word i holds codes (8 i + s, 8 i + s + 4); for
-// b = 2, pair p = 8 i + s holds codes (16 i + s, 16 i + s + 8).  The
-// activation pairs are permuted to match (xpair_nib).
-template <int B>
-__device__ __forceinline__ uint32_t pair_nib(const uint32_t (&w)[B], int p) {
-  static_assert(B == 2 || B == 4, "nibble pairs are for b = 2 and b = 4");
-  if constexpr (B == 4) return ((w[p >> 2] >> (4 * (p & 3))) & 0x000F000Fu) | 0x43004300u;
-  else return ((w[p >> 3] >> (2 * (p & 7))) & 0x00030003u) | 0x43004300u;
 }
 
 __device__ __forceinline__ uint32_t u4_comp(const uint4& v, int c) {
@@ -753,6 +719,56 @@ __device__ __forceinline__ void xpair_nib(const uint4 (&xv)[4], int j, uint32_t&
   b1 = __byte_perm(lo, hi, 0x7632);
 }
 
+// Pair p of a unit with its two codes as bf16 values code * 2^(c - 133): a
+// bf16 bit pattern whose high byte is zero is the integer in its low byte
+// times 2^-133 (the subnormals join the smallest binade without a gap), so
+// codes masked to bits [c, c + b) of the low byte of each 16-bit half need no
+// offset, no conversion and no zero point.  b = 4 and b = 2 take the pair
+// order of pair_nib (two codes 16 bits apart in one word; the upper byte's
+// codes after one shift by 8 per word), so c = pair_class<B>(p) varies with
+// p; b = 8 places bytes 2h, 2h + 1 of a word with one byte permute; the other
+// widths take consecutive codes at c = 0.
+template <int B>
+__host__ __device__ constexpr int pair_class(int p) {
+  return B == 4 ? 4 * (p & 1) : B == 2 ? 2 * (p & 3) : 0;
+}
+template <int B>
+__device__ __forceinline__ uint32_t pair_sub(const uint32_t (&w)[B], int p) {
+  if constexpr (B == 4) {
+    const uint32_t v = (p & 2) ? (w[p >> 2] >> 8) : w[p >> 2];
+    return v & (0x000F000Fu << pair_class<4>(p));
+  } else if constexpr (B == 2) {
+    const uint32_t v = (p & 4) ? (w[p >> 3] >> 8) : w[p >> 3];
+    return v & (0x00030003u << pair_class<2>(p));
+  } else if constexpr (B == 8) {
+    const int h = p & 1;
+    return __byte_perm(w[p >> 1], 0u, 0x4040 | (2 * h) | ((2 * h + 1) << 8));
+  } else if constexpr (B == 3 || B == 5) {
+    const int bit = 2 * B * p, wi = bit >> 5, sh = bit & 31;
+    const uint32_t x = sh + 2 * B <= 32 ? (w[wi] >> sh) : __funnelshift_r(w[wi], w[wi + 1], sh);
+    const uint32_t t = x & ((1u << (2 * B)) - 1u);
+    constexpr uint32_t mask = ((1u << B) - 1u) * 0x00010001u;
+    return (t * (1u + (1u << (16 - B)))) & mask;
+  } else {
+    return dq::code_at<B>(w, 2 * p) | (dq::code_at<B>(w, 2 * p + 1) << 16);
+  }
+}
+
+// bf16x2 (2^e, 2^e), e in [-126, 127].
+__device__ __forceinline__ uint32_t bf16x2_pow2(int e) { return static_cast<uint32_t>(e + 127) * 0x00800080u; }
+
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+// max(|a|, |b|) per half; the sign bit of the result is sign(a) ^ sign(b).
+__device__ __forceinline__ uint32_t bf16x2_maxabs(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t ld_ro_u16(const void* p) {
   unsigned short r;
   asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(r) : "l"(p));
@@ -770,9 +786,9 @@ constexpr int gemv_stage_bytes() {  // one warp's stage
 }
 
 template <int B, int RT, int S>
-constexpr int gemv_depth() {  // stages per warp: about 6 KiB of ring per warp, 2..8
-  constexpr int d = 6 * 1024 / gemv_stage_bytes<B, RT, 2>();
-  return d < 2 ? 2 : d > 8 ? 8 : d;
+constexpr int gemv_depth() {  // stages per warp: about 12 KiB of ring per warp, 3..8
+  constexpr int d = 12 * 1024 / gemv_stage_bytes<B, RT, 2>();
+  return d < 3 ? 3 : d > 8 ? 8 : d;
 }
 
 template <int B, int RT, int S>
@@ -806,7 +822,6 @@ __device__ __forceinline__ void gemv_tile(const GemvLayer& L, int M, int y_f32, 
   constexpr int kRowG = 16 * B;  // bytes of one row's group
   constexpr int kStage = gemv_stage_bytes<B, RT, GB>();
   constexpr bool kNib = B == 2 || B == 4;
-  constexpr bool kFold = B != 8;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = lane & 3, q = lane >> 2;
   const int G = K / kGroup;
@@ -864,6 +879,22 @@ __device__ __forceinline__ void gemv_tile(const GemvLayer& L, int M, int y_f32, 
     if (d < nb) issue(d, g0 + d * GB);
     cp_async_commit();
   }
+  // Activation fragments X[n][128 g + 32 t + 4 j .. + 3] (k-step j) of one
+  // group; loaded one group ahead, alternating between two register sets.
+  auto load_x = [&](int g, uint4 (&xv)[NT][4]) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int n = q + 8 * nt;
+      const uint16_t* xp = X + static_cast<int64_t>(n) * K + g * kGroup + 32 * t;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) xv[nt][v] = n < M ? ld_ro_v4(xp + 8 * v) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  // The first group's activations are in flight with the weights' first
+  // stages while the scales and zeros are staged.
+  constexpr bool kAhead = NT == 1;
+  uint4 xa[NT][4], xb[NT][4];
+  if (kAhead && ng > 0) load_x(g0, xa);
   // This warp's scales and zeros, (scale | zero << 16) per (row, group).
   // Each lane issues up to kSzBatch loads of each kind before its first
   // store, so a batch costs one memory latency rather than one per entry.
@@ -897,17 +928,6 @@ __device__ __forceinline__ void gemv_tile(const GemvLayer& L, int M, int y_f32, 
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[rt][nt][e] = 0.0f;
 
-  // Activation fragments X[n][128 g + 32 t + 4 j .. + 3] (k-step j) of one
-  // group; loaded one group ahead, alternating between two register sets.
-  auto load_x = [&](int g, uint4 (&xv)[NT][4]) {
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int n = q + 8 * nt;
-      const uint16_t* xp = X + static_cast<int64_t>(n) * K + g * kGroup + 32 * t;
-#pragma unroll
-      for (int v = 0; v < 4; ++v) xv[nt][v] = n < M ? ld_ro_v4(xp + 8 * v) : make_uint4(0u, 0u, 0u, 0u);
-    }
-  };
   auto group = [&](const uint8_t* st, int i, int gl, const uint4 (&xpre)[NT][4]) {
     // M <= 8: the fragments came one group ahead; M > 8: loaded here (two
     // register sets of 32 would spill next to two row tiles).
@@ -932,20 +952,23 @@ __device__ __forceinline__ void gemv_tile(const GemvLayer& L, int M, int y_f32, 
 #pragma unroll
         for (int rt = 0; rt < RT; ++rt) d[rt][nt][e] = 0.0f;
       }
-    uint32_t z2[RT][2];
-    float zf[RT][2];
-    if constexpr (!kFold) {
+    // The group's activation exponent: with 2^e <= max |x| < 2^(e + 1),
+    // E = 126 - e puts every x 2^E below 2^127 (clamped to [6, 127]: 2^(E - c)
+    // stays a normal bf16 for c <= 6, and 2^(133 - E) a normal binary32).
+    uint32_t xm = 0u;
 #pragma unroll
-      for (int rt = 0; rt < RT; ++rt)
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t z = sz[rt][h] >> 16;
-          z2[rt][h] = (0x4300u | z) * 0x00010001u;
-          zf[rt][h] = __uint_as_float(0x4B000000u | z);
-        }
-    }
+      for (int v = 0; v < 4; ++v)
+        xm = bf16x2_maxabs(bf16x2_maxabs(xm, xv[nt][v].x), bf16x2_maxabs(xv[nt][v].y,
+                           bf16x2_maxabs(xv[nt][v].z, xv[nt][v].w)));
+    xm &= 0x7FFF7FFFu;
+    xm = __reduce_max_sync(0xFFFFFFFFu, max(xm & 0xFFFFu, xm >> 16));
+    const int E = min(127, max(6, 126 - (static_cast<int>(xm >> 7) - 127)));
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
+      const int c0 = pair_class<B>(2 * j), c1 = pair_class<B>(2 * j + 1);
+      const uint32_t sc0 = bf16x2_pow2(E - c0), sc1 = bf16x2_pow2(E - c1);
       uint32_t b0[NT], b1[NT];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -955,54 +978,36 @@ __device__ __forceinline__ void gemv_tile(const GemvLayer& L, int M, int y_f32, 
           b0[nt] = (j & 1) ? xv[nt][j >> 1].z : xv[nt][j >> 1].x;
           b1[nt] = (j & 1) ? xv[nt][j >> 1].w : xv[nt][j >> 1].y;
         }
-        if constexpr (kFold)
-          mma_bf16_16816(dsum[nt], 0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u, b0[nt], b1[nt]);
+        b0[nt] = bf16x2_mul(b0[nt], sc0);
+        b1[nt] = bf16x2_mul(b1[nt], sc1);
+        // Sx = sum_k x_k 2^(E - 133) in the accumulator layout (A = 2^(c - 133)).
+        const uint32_t o0 = 0x00010001u << c0, o1 = 0x00010001u << c1;
+        mma_bf16_16816(dsum[nt], o0, o0, o1, o1, b0[nt], b1[nt]);
       }
 #pragma unroll
       for (int rt = 0; rt < RT; ++rt) {
-        uint32_t a0, a1, a2, a3;
-        if constexpr (kNib) {
-          a0 = pair_nib<B>(w[rt][0], 2 * j);
-          a1 = pair_nib<B>(w[rt][1], 2 * j);
-          a2 = pair_nib<B>(w[rt][0], 2 * j + 1);
-          a3 = pair_nib<B>(w[rt][1], 2 * j + 1);
-        } else if constexpr (kFold) {
-          a0 = pair_raw<B>(w[rt][0], 2 * j);
-          a1 = pair_raw<B>(w[rt][1], 2 * j);
-          a2 = pair_raw<B>(w[rt][0], 2 * j + 1);
-          a3 = pair_raw<B>(w[rt][1], 2 * j + 1);
-        } else {
-          a0 = pair_of<B>(w[rt][0], z2[rt][0], zf[rt][0], 2 * j);
-          a1 = pair_of<B>(w[rt][1], z2[rt][1], zf[rt][1], 2 * j);
-          a2 = pair_of<B>(w[rt][0], z2[rt][0], zf[rt][0], 2 * j + 1);
-          a3 = pair_of<B>(w[rt][1], z2[rt][1], zf[rt][1], 2 * j + 1);
-        }
+        const uint32_t a0 = pair_sub<B>(w[rt][0], 2 * j);
+        const uint32_t a1 = pair_sub<B>(w[rt][1], 2 * j);
+        const uint32_t a2 = pair_sub<B>(w[rt][0], 2 * j + 1);
+        const uint32_t a3 = pair_sub<B>(w[rt][1], 2 * j + 1);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(d[rt][nt], a0, a1, a2, a3, b0[nt], b1[nt]);
       }
     }
+    // y += s 2^(133 - E) (D - z Sx): D = sum_k q x 2^(E - 133).
+    const float pw = __uint_as_float(static_cast<uint32_t>(260 - E) << 23);
 #pragma unroll
     for (int rt = 0; rt < RT; ++rt) {
-      const float s0 = __half2float(__ushort_as_half(static_cast<uint16_t>(sz[rt][0] & 0xFFFFu)));
-      const float s1 = __half2float(__ushort_as_half(static_cast<uint16_t>(sz[rt][1] & 0xFFFFu)));
-      if constexpr (kFold) {
-        const float zb0 = -static_cast<float>(128u + (sz[rt][0] >> 16));
-        const float zb1 = -static_cast<float>(128u + (sz[rt][1] >> 16));
+      const float s0 = __half2float(__ushort_as_half(static_cast<uint16_t>(sz[rt][0] & 0xFFFFu))) * pw;
+      const float s1 = __half2float(__ushort_as_half(static_cast<uint16_t>(sz[rt][1] & 0xFFFFu))) * pw;
+      const float zb0 = -static_cast<float>(sz[rt][0] >> 16);
+      const float zb1 = -static_cast<float>(sz[rt][1] >> 16);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          acc[rt][nt][0] = fmaf(s0, fmaf(zb0, dsum[nt][0], d[rt][nt][0]), acc[rt][nt][0]);
-          acc[rt][nt][1] = fmaf(s0, fmaf(zb0, dsum[nt][1], d[rt][nt][1]), acc[rt][nt][1]);
-          acc[rt][nt][2] = fmaf(s1, fmaf(zb1, dsum[nt][2], d[rt][nt][2]), acc[rt][nt][2]);
-          acc[rt][nt][3] = fmaf(s1, fmaf(zb1, dsum[nt][3], d[rt][nt][3]), acc[rt][nt][3]);
-        }
-      } else {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          acc[rt][nt][0] = fmaf(s0, d[rt][nt][0], acc[rt][nt][0]);
-          acc[rt][nt][1] = fmaf(s0, d[rt][nt][1], acc[rt][nt][1]);
-          acc[rt][nt][2] = fmaf(s1, d[rt][nt][2], acc[rt][nt][2]);
-          acc[rt][nt][3] = fmaf(s1, d[rt][nt][3], acc[rt][nt][3]);
-        }
+      for (int nt = 0; nt < NT; ++nt) {
+        acc[rt][nt][0] = fmaf(s0, fmaf(zb0, dsum[nt][0], d[rt][nt][0]), acc[rt][nt][0]);
+        acc[rt][nt][1] = fmaf(s0, fmaf(zb0, dsum[nt][1], d[rt][nt][1]), acc[rt][nt][1]);
+        acc[rt][nt][2] = fmaf(s1, fmaf(zb1, dsum[nt][2], d[rt][nt][2]), acc[rt][nt][2]);
+        acc[rt][nt][3] = fmaf(s1, fmaf(zb1, dsum[nt][3], d[rt][nt][3]), acc[rt][nt][3]);
       }
     }
   };
@@ -1011,9 +1016,6 @@ __device__ __forceinline__ void gemv_tile(const GemvLayer& L, int M, int y_f32, 
   // while xb is loaded for the second, which loads xa for the next stage's
   // first.
   static_assert(GB == 2, "the activation double buffer alternates within a stage");
-  constexpr bool kAhead = NT == 1;
-  uint4 xa[NT][4], xb[NT][4];
-  if (kAhead && ng > 0) load_x(g0, xa);
   for (int bi = 0; bi < nb; ++bi) {
     const int nx = bi + D - 1;
     if (nx < nb) issue(nx % D, g0 + nx * GB);
@@ -1133,8 +1135,6 @@ int resident_ctas() {
   return sms * kCtasPerSm;
 }
 
-size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
-
 template <int B, int NT, int GS>
 cudaError_t launch_cfg(const uint16_t* X, int M, int N, int K, const uint32_t* packed,
                        const uint16_t* scales, const uint8_t* zeros, void* Y, bool y_f32,
@@ -1246,22 +1246,45 @@ cudaError_t launch_gemv_cfg(const uint16_t* X, int M, int N, int K, const uint32
   return cudaLaunchKernelEx(&cfg, kern, L, M, y_f32 ? 1 : 0);
 }
 
+// Tile shape of a GEMV launch over `rows` weight rows with G groups each
+// (measured on this B200 over the Qwen3-8B block's layers and 8192 x 8192,
+// graph-timed, M = 1, 4, 16):
+//  * RT: the CTAs of a launch run concurrently, so an SM's time follows the
+//    rows it gets, ceil(tiles / SMs) * 16 RT.  Two m16 tiles per warp share
+//    the per-group activation work, so RT = 2 unless one tile per warp puts
+//    at least a fifth fewer rows on the busiest SM (or rt2 is not allowed).
+//  * S (warps splitting K): 16 when the tiles leave SMs idle and K is long,
+//    4 once there are two tiles per SM or more, else 8.
+struct GemvShape {
+  int rt, s;
+};
+GemvShape gemv_shape(int64_t rows, int G, bool rt2, int sms) {
+  const int64_t t1 = (rows + 15) / 16, t2 = (rows + 31) / 32;
+  const int64_t w1 = (t1 + sms - 1) / sms, w2 = 2 * ((t2 + sms - 1) / sms);
+  const int rt = (!rt2 || 5 * w1 < 4 * w2) ? 1 : 2;
+  const int64_t tiles = rt == 1 ? t1 : t2;
+  int s = 8;
+  if (tiles < sms && G >= 32) s = 16;
+  else if (tiles >= 2 * sms || G < 16) s = 4;
+  return {rt, s};
+}
+
+int device_sms() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
 template <int B, int NT, int RT>
-cudaError_t launch_gemv_nt(const uint16_t* X, int M, int N, int K, const uint32_t* packed,
+cudaError_t launch_gemv_rt(int s, const uint16_t* X, int M, int N, int K, const uint32_t* packed,
                            const uint16_t* scales, const uint8_t* zeros, void* Y, bool y_f32,
                            cudaStream_t stream) {
-  // K splits per row tile: 4 warps per tile once the layer has about 16
-  // warps' worth of 16-row blocks per SM, more splits for layers with fewer
-  // (measured on this B200 over the Qwen3-8B and 8192 x 8192 layers).
-  const int tiles = (N + 16 * RT - 1) / (16 * RT);
-  const int G = K / kGroup;
+  // A shape whose rings do not fit falls back to fewer warps.
   if constexpr (gemv_fits<B, RT, 16>()) {
-    if ((NT == 2 ? tiles : tiles * RT) < 148 && G >= 32)
-      return launch_gemv_cfg<B, NT, RT, 16>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
+    if (s == 16) return launch_gemv_cfg<B, NT, RT, 16>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
   }
   if constexpr (gemv_fits<B, RT, 8>()) {
-    if (tiles * RT < 600 && G >= 16)
-      return launch_gemv_cfg<B, NT, RT, 8>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
+    if (s >= 8) return launch_gemv_cfg<B, NT, RT, 8>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
   }
   return launch_gemv_cfg<B, NT, RT, 4>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
 }
@@ -1270,21 +1293,15 @@ template <int B>
 cudaError_t launch_gemv_b(const uint16_t* X, int M, int N, int K, const uint32_t* packed,
                           const uint16_t* scales, const uint8_t* zeros, void* Y, bool y_f32,
                           cudaStream_t stream) {
+  // At M <= 8, b = 7 and 8, the doubled unit registers of RT = 2 cost more
+  // than the shared activation work saves.
+  const GemvShape sh = gemv_shape(N, K / kGroup, M > 8 || B <= 6, device_sms());
   if (M <= 8) {
-    // Two m16 tiles per warp also pay at M <= 8 for b <= 6, where the
-    // per-group activation and scale work is a larger share (measured; at
-    // b = 7, 8 the doubled unit registers cost more than they save).
-    if constexpr (B <= 6) {
-      if ((N + 31) / 32 >= 128)
-        return launch_gemv_nt<B, 1, 2>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
-    }
-    return launch_gemv_nt<B, 1, 1>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
+    if (sh.rt == 2) return launch_gemv_rt<B, 1, 2>(sh.s, X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
+    return launch_gemv_rt<B, 1, 1>(sh.s, X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
   }
-  // Two m16 tiles per warp share each activation fragment; worth it once the
-  // layer has about one 32-row tile per SM.
-  if ((N + 31) / 32 >= 128)
-    return launch_gemv_nt<B, 2, 2>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
-  return launch_gemv_nt<B, 2, 1>(X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
+  if (sh.rt == 2) return launch_gemv_rt<B, 2, 2>(sh.s, X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
+  return launch_gemv_rt<B, 2, 1>(sh.s, X, M, N, K, packed, scales, zeros, Y, y_f32, stream);
 }
 
 }  // namespace
@@ -1375,21 +1392,15 @@ cudaError_t launch_group_cfg(const GemvLayer* layers, int count, int M, bool y_f
 
 // The same shape rules as a single layer, applied to the group's totals.
 template <int NT, int RT>
-cudaError_t launch_group_rt(const GemvLayer* layers, int count, int M, bool y_f32,
+cudaError_t launch_group_rt(int s, const GemvLayer* layers, int count, int M, bool y_f32,
                             cudaStream_t stream) {
-  int tiles = 0, gmin = 1 << 30;
-  for (int i = 0; i < count; ++i) {
-    tiles += (layers[i].N + 16 * RT - 1) / (16 * RT);
-    const int G = layers[i].K / kGroup;
-    gmin = G < gmin ? G : gmin;
-  }
   bool fits = false;
   cudaError_t e = cudaSuccess;
-  if ((NT == 2 ? tiles : tiles * RT) < 148 && gmin >= 32) {
+  if (s == 16) {
     e = launch_group_cfg<NT, RT, 16>(layers, count, M, y_f32, stream, &fits);
     if (fits || e != cudaSuccess) return e;
   }
-  if (tiles * RT < 600 && gmin >= 16) {
+  if (s >= 8) {
     e = launch_group_cfg<NT, RT, 8>(layers, count, M, y_f32, stream, &fits);
     if (fits || e != cudaSuccess) return e;
   }
@@ -1417,14 +1428,17 @@ cudaError_t launch_gemm_gemv_group(const GemvCall* calls, int count, int64_t M, 
     bmax = c.bits > bmax ? c.bits : bmax;
   }
   const int m = static_cast<int>(M);
-  // Two m16 tiles per warp on the rules of the single-layer launch.
+  // The single-layer shape rule over all the layers' rows (each layer's
+  // tiles are whole; the shortest K decides the warp split).
+  int gmin = 1 << 30;
+  for (int i = 0; i < count; ++i) gmin = layers[i].K / kGroup < gmin ? layers[i].K / kGroup : gmin;
+  const GemvShape sh = gemv_shape(rows, gmin, m > 8 || bmax <= 6, device_sms());
   if (m <= 8) {
-    if (bmax <= 6 && (rows + 31) / 32 >= 128)
-      return launch_group_rt<1, 2>(layers, count, m, y_f32, stream);
-    return launch_group_rt<1, 1>(layers, count, m, y_f32, stream);
+    if (sh.rt == 2) return launch_group_rt<1, 2>(sh.s, layers, count, m, y_f32, stream);
+    return launch_group_rt<1, 1>(sh.s, layers, count, m, y_f32, stream);
   }
-  if ((rows + 31) / 32 >= 128) return launch_group_rt<2, 2>(layers, count, m, y_f32, stream);
-  return launch_group_rt<2, 1>(layers, count, m, y_f32, stream);
+  if (sh.rt == 2) return launch_group_rt<2, 2>(sh.s, layers, count, m, y_f32, stream);
+  return launch_group_rt<2, 1>(sh.s, layers, count, m, y_f32, stream);
 }
 
 // ---------------------------------------------------------------------------
