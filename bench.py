@@ -466,7 +466,7 @@ def run_slq(args, rank, world, local_rank):
             },
             "roofline": {
                 "bound": "hbm",
-                "kernel": "gemm_gemv_group_kernel / gemm_gemv_kernel<b> (split-K GEMV: packed W streamed by cp.async through per-warp shared-memory rings, dequantized in registers into mma.sync A fragments, zero point folded out for b<=7, fp32 group-scaled accumulate, deterministic in-CTA split-K; M<=16)",
+                "kernel": "gemm_gemv_group_kernel / gemm_gemv_kernel<b> (split-K GEMV: packed W streamed by cp.async through per-warp shared-memory rings; the codes masked in place are exact subnormal bf16 mma.sync A fragments, the activations scaled by 2^(E-c) per group, the zero point folded out through a constant-A mma, fp32 group-scaled accumulate, deterministic in-CTA split-K; M<=16)",
                 "achieved": round(achieved, 1),
                 "peak": hbm_peak,
                 "unit": "GB/s",
