@@ -51,7 +51,8 @@ typedef enum { SLQ_DTYPE_BF16 = 0, SLQ_DTYPE_F32 = 1 } slq_dtype;
 enum {
   SLQ_FLAG_NONFINITE = 1u,      /* a weight was inf or NaN: that group's output is unspecified */
   SLQ_FLAG_SCALE_OVERFLOW = 2u, /* a group's range exceeded fp16: scale stored as 65504 */
-  SLQ_FLAG_TIMEOUT = 4u         /* a bounded on-chip wait gave up; outputs are unspecified */
+  SLQ_FLAG_TIMEOUT = 4u,        /* a bounded on-chip wait gave up; outputs are unspecified */
+  SLQ_FLAG_NOT_POSITIVE_DEFINITE = 8u /* slq_gptq: a Cholesky pivot was not positive; outputs unspecified */
 };
 
 /* GEMM kernel choice for slq_gemm_ex.  Every kernel forms exact bf16 values
@@ -339,6 +340,50 @@ int slq_ear_kl_topk_max(void);
 slq_status slq_grid_noise(const void *W_bf16, int64_t N, int64_t K, int bits,
                           float *gamma, float *sse_asym, float *sse_sym,
                           uint32_t *flags, void *stream);
+
+/*
+ * slq_gptq -- GPTQ encode of W with calibration rows X into the same format
+ * as slq_quantize (asymmetric INT-`bits`, groups of 128 along K, fp16 scales,
+ * uint8 zeros, LSB-first packed codes).
+ *
+ * Source: the pages' encoder is layer-wise GPTQ at every b with asymmetric
+ * INT, group size 128 (GitHub README, "Pipeline" and "1. Quantize"); GPTQ as
+ * published by Frantar et al.  Readings where the pages are silent:
+ * H = X^T X in binary64; an input column that is always zero gets H_kk = 1
+ * and its weights set to 0; damping H += damp * mean(diag H) * I; columns in
+ * natural order; a group's scale and zero come from its current, already
+ * updated weights at its first column, by slq_quantize's rules; weights are
+ * carried in binary64 and rounded to binary32 for each encode; with U the
+ * upper Cholesky factor of H^-1 (H^-1 = U^T U), fixing column k with
+ * dequantized value d moves every later column j by -(w_k - d) / U_kk * U_kj.
+ * Every value is formed by the same sequence of correctly rounded binary64
+ * (binary32 for the encode) operations as that definition, so the outputs do
+ * not depend on the launch shape.
+ *
+ * W_bf16     [N, K] row-major bf16, device.  N >= 0 (0 writes nothing).
+ * K          a positive multiple of 128, at most 16384.
+ * bits       2..8.
+ * X_bf16     [T, K] row-major bf16, device: calibration rows, T >= 1.
+ * damp       finite, >= 0 (the pages' runs use 0.01).
+ * packed, scales_f16, zeros   outputs as for slq_quantize.
+ * workspace  device, 16-byte aligned, slq_gptq_workspace_bytes(N, K) bytes
+ *            or more, owned by the caller, not read across calls.
+ * flags      device uint32 or NULL: SLQ_FLAG_NONFINITE, _SCALE_OVERFLOW as
+ *            for slq_quantize; SLQ_FLAG_NOT_POSITIVE_DEFINITE when the damped
+ *            H (or its inverse) has a non-positive Cholesky pivot.
+ * Runs about 2 K + 2 K/128 + 8 launches on `stream`.  Errors:
+ * SLQ_ERR_INVALID_ARGUMENT for sizes, alignment, a short workspace or
+ * overlapping buffers, before any launch; SLQ_ERR_CUDA for a failed launch.
+ */
+slq_status slq_gptq(const void *W_bf16, int64_t N, int64_t K, int bits,
+                    const void *X_bf16, int64_t T, double damp, uint32_t *packed,
+                    void *scales_f16, uint8_t *zeros, void *workspace,
+                    size_t workspace_bytes, uint32_t *flags, void *stream);
+
+/* Workspace bytes slq_gptq needs for an [N, K] layer (0 for invalid sizes):
+ * three K x K binary64 matrices, the layer in binary64, and 128 binary64
+ * errors per row. */
+size_t slq_gptq_workspace_bytes(int64_t N, int64_t K);
 
 #ifdef __cplusplus
 }

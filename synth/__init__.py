@@ -71,6 +71,19 @@ def activations(M: int, K: int, seed: int = SEED_X) -> np.ndarray:
     return to_bf16_bits(rng.standard_normal((M, K)))
 
 
+def calibration(T: int, K: int, seed: int = SEED_X, rho: float = 0.9) -> np.ndarray:
+    """Calibration rows [T, K] bf16 bits whose neighbouring inputs are
+    correlated: x_k = rho x_{k-1} + sqrt(1 - rho^2) z_k, z ~ N(0, 1) (standing
+    in for the pages' FineWeb-Edu calibration tokens)."""
+    rng = np.random.default_rng(seed)
+    z = rng.standard_normal((T, K))
+    x = np.empty_like(z)
+    x[:, 0] = z[:, 0]
+    for k in range(1, K):
+        x[:, k] = rho * x[:, k - 1] + np.sqrt(1 - rho**2) * z[:, k]
+    return to_bf16_bits(x)
+
+
 def logits(T: int, V: int, seed: int = SEED_LOGITS, noise_seed: int = SEED_LOGIT_NOISE,
            std: float = 3.0, peak: float = 6.0, noise_std: float = 0.05):
     """(reference, quantized) logit rows, each [T, V] bf16 bits."""

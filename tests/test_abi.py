@@ -225,3 +225,22 @@ def test_grid_noise_validation():
         assert call(**bad) == slq.SLQ_ERR_INVALID_ARGUMENT, bad
     assert call(N=0) == slq.SLQ_OK
     assert call() in (slq.SLQ_OK, slq.SLQ_ERR_UNSUPPORTED_DEVICE)
+
+
+def test_gptq_validation():
+    need = slq.gptq_workspace_bytes(64, 256)
+    assert need == L.slq_gptq_workspace_bytes(64, 256) and need > 3 * 256 * 256 * 8
+    assert L.slq_gptq_workspace_bytes(64, 100) == 0
+    assert L.slq_gptq_workspace_bytes(64, 16384 + 128) == 0
+
+    def call(W=FAKE, N=64, K=256, bits=4, X=FAKE + (1 << 24), T=32, damp=0.01, p=FAKE + (2 << 24),
+             s=FAKE + (3 << 24), z=FAKE + (4 << 24), ws=FAKE + (5 << 24), wsb=need, flags=None):
+        return L.slq_gptq(W, N, K, bits, X, T, damp, p, s, z, ws, wsb, flags, None)
+
+    for bad in [dict(N=-1), dict(K=200), dict(K=16384 + 128), dict(bits=9), dict(T=0), dict(damp=-1.0),
+                dict(damp=float("nan")), dict(damp=float("inf")), dict(W=None), dict(X=None),
+                dict(ws=None), dict(wsb=need - 1), dict(ws=FAKE + (5 << 24) + 8), dict(p=FAKE + 2),
+                dict(p=FAKE + 16)]:                    # output overlaps W
+        assert call(**bad) == slq.SLQ_ERR_INVALID_ARGUMENT, bad
+    assert call(N=0) == slq.SLQ_OK
+    assert call() in (slq.SLQ_OK, slq.SLQ_ERR_UNSUPPORTED_DEVICE)

@@ -38,6 +38,7 @@ SLQ_DTYPE_F32 = 1
 SLQ_FLAG_NONFINITE = 1
 SLQ_FLAG_SCALE_OVERFLOW = 2
 SLQ_FLAG_TIMEOUT = 4
+SLQ_FLAG_NOT_POSITIVE_DEFINITE = 8
 
 SLQ_GEMM_AUTO = 0
 SLQ_GEMM_DECODE = 1
@@ -97,6 +98,10 @@ _lib.slq_ear_kl_topk_max.argtypes = []
 _lib.slq_ear_kl_topk_max.restype = _I
 _lib.slq_grid_noise.argtypes = [_P, _I64, _I64, _I, _P, _P, _P, _P, _P]
 _lib.slq_grid_noise.restype = _I
+_lib.slq_gptq.argtypes = [_P, _I64, _I64, _I, _P, _I64, ctypes.c_double, _P, _P, _P, _P, _SZ, _P, _P]
+_lib.slq_gptq.restype = _I
+_lib.slq_gptq_workspace_bytes.argtypes = [_I64, _I64]
+_lib.slq_gptq_workspace_bytes.restype = _SZ
 
 
 def lib() -> ctypes.CDLL:
@@ -476,3 +481,40 @@ def grid_noise(W, bits: int, flags=None, stream=None):
         _check(_lib.slq_grid_noise(_ptr(W), N, K, bits, _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]),
                                    _ptr(flags), _stream_ptr(stream, dev)), "slq_grid_noise")
     return tuple(outs)
+
+
+def gptq_workspace_bytes(N: int, K: int) -> int:
+    return int(_lib.slq_gptq_workspace_bytes(N, K))
+
+
+def gptq(W, X, bits: int, damp: float = 0.01, out: QuantizedWeight | None = None, flags=None,
+         stream=None, workspace=None) -> QuantizedWeight:
+    """GPTQ encode (slq_gptq) of a [N, K] bf16 CUDA tensor with [T, K] bf16
+    calibration rows X into the packed format of quantize().  `workspace` (a
+    uint8 CUDA tensor of gptq_workspace_bytes(N, K) bytes or more) is
+    allocated for the call when not given."""
+    import torch
+    _require(W, "W", (torch.bfloat16,), ndim=2)
+    N, K = W.shape
+    _require_bits_k(bits, K)
+    _require(X, "X", (torch.bfloat16,), ndim=2)
+    if X.shape[1] != K:
+        raise ValueError(f"X: {tuple(X.shape)}, expected [T, {K}]")
+    if out is not None:
+        _require_weight(out, "out")
+        if (out.N, out.K, out.bits) != (N, K, bits):
+            raise ValueError(f"out: a ({out.N}, {out.K}, {out.bits}-bit) layer, "
+                             f"expected ({N}, {K}, {bits}-bit)")
+    _require_flags(flags)
+    if workspace is not None:
+        _require(workspace, "workspace", (torch.uint8,))
+    dev = _require_cuda(W=W, X=X, flags=flags, workspace=workspace,
+                        out=None if out is None else out.packed)
+    with _on(dev):
+        q = out if out is not None else empty_quantized(N, K, bits, dev)
+        need = gptq_workspace_bytes(N, K)
+        ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8, device=dev)
+        _check(_lib.slq_gptq(_ptr(W), N, K, bits, _ptr(X), X.shape[0], float(damp), _ptr(q.packed),
+                             _ptr(q.scales), _ptr(q.zeros), _ptr(ws), ws.numel(), _ptr(flags),
+                             _stream_ptr(stream, dev)), "slq_gptq")
+    return q

@@ -37,6 +37,7 @@ struct SmemAttr {
 constexpr uint32_t kFlagNonfinite = 1u;
 constexpr uint32_t kFlagScaleOverflow = 2u;
 constexpr uint32_t kFlagTimeout = 4u;
+constexpr uint32_t kFlagNotPositiveDefinite = 8u;
 
 cudaError_t launch_quantize(const uint16_t* W, int64_t N, int64_t K, int bits,
                             uint32_t* packed, uint16_t* scales, uint8_t* zeros,
@@ -119,5 +120,12 @@ cudaError_t launch_ear_kl_topk(const uint16_t* a, const uint16_t* b, int64_t T, 
 // continuous b-bit grids; outputs [N, K / 128] fp32.
 cudaError_t launch_grid_noise(const uint16_t* W, int64_t N, int64_t K, int bits, float* gamma,
                               float* sse_asym, float* sse_sym, uint32_t* flags, cudaStream_t stream);
+
+// GPTQ encode (binary64, the definition's operation order); workspace of
+// gptq_workspace_bytes(N, K) bytes, 16-byte aligned.
+size_t gptq_workspace_bytes(int64_t N, int64_t K);
+cudaError_t launch_gptq(const uint16_t* W, int64_t N, int64_t K, int bits, const uint16_t* X, int64_t T,
+                        double damp, uint32_t* packed, uint16_t* scales, uint8_t* zeros, void* workspace,
+                        uint32_t* flags, cudaStream_t stream);
 
 }  // namespace slq

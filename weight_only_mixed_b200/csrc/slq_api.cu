@@ -344,4 +344,38 @@ slq_status slq_grid_noise(const void* W_bf16, int64_t N, int64_t K, int bits, fl
                                           static_cast<cudaStream_t>(stream)));
 }
 
+size_t slq_gptq_workspace_bytes(int64_t N, int64_t K) {
+  if (N < 0 || N > kMaxDim || !valid_k(K) || K > 16384 || !product_ok(N, K)) return 0;
+  return slq::gptq_workspace_bytes(N, K);
+}
+
+slq_status slq_gptq(const void* W_bf16, int64_t N, int64_t K, int bits, const void* X_bf16, int64_t T,
+                    double damp, uint32_t* packed, void* scales_f16, uint8_t* zeros, void* workspace,
+                    size_t workspace_bytes, uint32_t* flags, void* stream) {
+  if (N < 0 || N > kMaxDim || !valid_k(K) || K > 16384 || !valid_bits(bits) || !product_ok(N, K))
+    return SLQ_ERR_INVALID_ARGUMENT;
+  if (T < 1 || T > kMaxDim || !product_ok(T, K) || !std::isfinite(damp) || !(damp >= 0.0))
+    return SLQ_ERR_INVALID_ARGUMENT;
+  if (N == 0) return SLQ_OK;
+  if (!W_bf16 || !X_bf16 || !packed || !scales_f16 || !zeros || !workspace)
+    return SLQ_ERR_INVALID_ARGUMENT;
+  const size_t need = slq::gptq_workspace_bytes(N, K);
+  if (workspace_bytes < need) return SLQ_ERR_INVALID_ARGUMENT;
+  if (!aligned(W_bf16, 2) || !aligned(X_bf16, 2) || !aligned(packed, 4) || !aligned(scales_f16, 2) ||
+      !aligned(workspace, 16) || (flags && !aligned(flags, 4)))
+    return SLQ_ERR_INVALID_ARGUMENT;
+  const int64_t G = K / slq::kGroup;
+  const Range ins[2] = {range_of(W_bf16, N * K * 2), range_of(X_bf16, T * K * 2)};
+  const Range outs[5] = {range_of(packed, N * K * bits / 8), range_of(scales_f16, N * G * 2),
+                         range_of(zeros, N * G), range_of(flags, flags ? 4 : 0),
+                         range_of(workspace, static_cast<int64_t>(need))};
+  if (!disjoint(outs, 5, ins, 2)) return SLQ_ERR_INVALID_ARGUMENT;
+  const slq_status dev = check_device();
+  if (dev != SLQ_OK) return dev;
+  return from_cuda(slq::launch_gptq(static_cast<const uint16_t*>(W_bf16), N, K, bits,
+                                    static_cast<const uint16_t*>(X_bf16), T, damp, packed,
+                                    static_cast<uint16_t*>(scales_f16), zeros, workspace, flags,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"
