@@ -31,6 +31,7 @@ timed ones; with --graph the K calls replay as one CUDA graph) and prints
   eartopk:T:V:tau:K         one top-K EAR/KL reduction
   quantize:N:K:b            one quantize+pack
   gridnoise:N:K:b           one grid-noise pass (gamma, asymmetric and symmetric SSE)
+  gptq:N:K:T:b              one GPTQ encode of an [N, K] layer with T calibration rows
 
 --impl reference times the CPU oracle (the plain reference implementation
 of the same arithmetic) on a bounded sample of the same workload, on the
@@ -73,6 +74,10 @@ def weight_bytes(N, K, bits):
 
 
 BLOCK_BYTES = sum(weight_bytes(N, K, b) for _, N, K, b in QWEN3_8B_BLOCK)
+
+# GPTQ rows: the oracle's timed sample, and a 4096 x 4096 projection with the
+# pages' 512 calibration rows per layer order of magnitude.
+GPTQ_SHAPES = [(256, 1024, 256, 4), (4096, 4096, 512, 4)]
 
 
 def load_peaks():
@@ -699,6 +704,18 @@ def other_rows(args, slq, synth, torch, dev, stream, hbm_peak, tc_peak, rank):
                                           "us": round(ms * 1e3, 1), "ear_mean": round(em.item(), 6),
                                           "kl_mean": round(km.item(), 7)}
     del a, bq
+
+    # GPTQ encode of one layer (slq_gptq: H, factorizations, column encode),
+    # on the oracle's sample shape and on a 4096 x 4096 projection.
+    for (N, K, T, b) in GPTQ_SHAPES:
+        W = synth.weights_torch(N, K, seed=800 + N, device=dev)
+        X = torch.from_numpy(synth.calibration(T, K, seed=801 + K).view(np.int16)).to(dev).view(torch.bfloat16)
+        out = slq.empty_quantized(N, K, b, dev)
+        ws = torch.empty(slq.gptq_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
+        slq.gptq(W, X, b, out=out, workspace=ws, stream=stream)
+        ms = time_ms(torch, stream, lambda: slq.gptq(W, X, b, out=out, workspace=ws, stream=stream), 3, warm=1)
+        rows[f"gptq_{N}x{K}_T{T}_b{b}"] = {"ms": round(ms, 2), "launches": 2 * K + 2 * (K // 128) + 8}
+        del W, X, out, ws
     return rows
 
 
@@ -768,6 +785,14 @@ def _oracle_job_prepared(job, barrier, queue):
                 oracle.quantize(w, b)
                 nb += w.size * 2 + weight_bytes(w.shape[0], w.shape[1], b)
             return nb
+    elif kind == "gptq":
+        _, N, K, T, b = job
+        w = synth.weights(N, K, seed=800 + N)
+        x = synth.calibration(T, K, seed=801 + K)
+
+        def run():
+            oracle.gptq(w, x, b)
+            return 1  # layers
     else:
         _, tokens, V, seed = job
         a, bq = synth.logits(tokens, V, seed=seed, noise_seed=seed + 1)
@@ -811,6 +836,10 @@ def oracle_rates(rows_per_layer: int, all_cores: bool):
     for name, job in jobs.items():
         nb, t0, t1 = _oracle_job_prepared(job, None, None)
         out[f"{name}_1core"] = nb / (t1 - t0) / 1e9
+    # GPTQ: seconds per layer on one core (its factorizations are not split
+    # over rows, so there is no all-core form of the same job).
+    _, t0, t1 = _oracle_job_prepared(("gptq",) + GPTQ_SHAPES[0], None, None)
+    out["gptq_1core_s"] = t1 - t0
     if all_cores and cores > 1:
         for name, job in jobs.items():
             par = [job if name != "ear" else _ear_job(8, k) for k in range(cores)]
@@ -831,9 +860,11 @@ def cpu_baseline(args):
         "sample": (f"decode GEMM of the Qwen3-8B block at M in {{1,4,16}}: the first {args.cpu_rows} output rows of "
                    f"each of the 7 projections per job, one job on 1 core and one job per core on {cores} spawned "
                    f"processes (os.sched_getaffinity) started together; quantize+pack: 64 rows of each projection per "
-                   f"job; EAR/KL: 8 tokens x 151936 per job (binary64 scalar C oracle, unchanged)"),
+                   f"job; EAR/KL: 8 tokens x 151936 per job; GPTQ: one {GPTQ_SHAPES[0][0]} x {GPTQ_SHAPES[0][1]} layer with "
+                   f"{GPTQ_SHAPES[0][2]} calibration rows at b = {GPTQ_SHAPES[0][3]} on one core (binary64 scalar C "
+                   f"oracle, unchanged)"),
         "single_core": {"gemm_GBps": r(rates["gemm_1core"]), "quantize_GBps": r(rates["quantize_1core"]),
-                        "ear_kl_GBps": r(rates["ear_1core"])},
+                        "ear_kl_GBps": r(rates["ear_1core"]), "gptq_s_per_layer": r(rates["gptq_1core_s"])},
         "all_cores": None if not allc else {"cores": cores, "gemm_GBps": r(rates["gemm_allcore"]),
                                             "quantize_GBps": r(rates["quantize_allcore"]),
                                             "ear_kl_GBps": r(rates["ear_allcore"])},
@@ -952,6 +983,16 @@ def run_case(args):
         def fn():
             slq.quantize(W, b, out=q, stream=stream)
         per_call = 1
+    elif kind == "gptq":
+        N, K, T, b = vals
+        W = synth.weights_torch(N, K, device=dev)
+        X = torch.from_numpy(synth.calibration(T, K).view(np.int16)).to(dev).view(torch.bfloat16)
+        out = slq.empty_quantized(N, K, b, dev)
+        ws = torch.empty(slq.gptq_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
+
+        def fn():
+            slq.gptq(W, X, b, out=out, workspace=ws, stream=stream)
+        per_call = 2 * K + 2 * (K // 128) + 8
     elif kind == "gridnoise":
         N, K, b = vals
         W = synth.weights_torch(N, K, device=dev)

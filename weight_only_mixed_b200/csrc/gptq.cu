@@ -122,6 +122,9 @@ __global__ void __launch_bounds__(256) chol_col_kernel(double* __restrict__ A, i
   const double* colj = A;  // element (r, k) at A[k K + r]
   double d = A[static_cast<int64_t>(j) * K + j];
   double v = A[static_cast<int64_t>(j) * K + i];
+  // Unrolled so that the loads of several steps are in flight: the chains
+  // themselves (d and v, in k order) are unchanged.
+#pragma unroll 8
   for (int k = 0; k < j; ++k) {
     const double ljk = colj[static_cast<int64_t>(k) * K + j];
     d = __dsub_rn(d, __dmul_rn(ljk, ljk));
@@ -165,6 +168,7 @@ __global__ void __launch_bounds__(128) tri_inverse_kernel(const double* __restri
     const double* li = Lr + static_cast<int64_t>(i) * K + c;  // L_{i, c + s}
     double v = i == c ? 1.0 : 0.0;
     const int n = i - c;
+#pragma unroll 8
     for (int s = 0; s < n; ++s) v = __dsub_rn(v, __dmul_rn(li[s], Dg[static_cast<int64_t>(s) * K + c]));
     Dg[static_cast<int64_t>(n) * K + c] = __ddiv_rn(v, Lr[static_cast<int64_t>(i) * K + i]);
   }
