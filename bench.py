@@ -714,7 +714,7 @@ def other_rows(args, slq, synth, torch, dev, stream, hbm_peak, tc_peak, rank):
         ws = torch.empty(slq.gptq_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
         slq.gptq(W, X, b, out=out, workspace=ws, stream=stream)
         ms = time_ms(torch, stream, lambda: slq.gptq(W, X, b, out=out, workspace=ws, stream=stream), 3, warm=1)
-        rows[f"gptq_{N}x{K}_T{T}_b{b}"] = {"ms": round(ms, 2), "launches": 2 * K + 2 * (K // 128) + 8}
+        rows[f"gptq_{N}x{K}_T{T}_b{b}"] = {"ms": round(ms, 2), "launches": 6 * (K // 32) + 2 * (K // 128) + 3}
         del W, X, out, ws
     return rows
 
@@ -992,7 +992,7 @@ def run_case(args):
 
         def fn():
             slq.gptq(W, X, b, out=out, workspace=ws, stream=stream)
-        per_call = 2 * K + 2 * (K // 128) + 8
+        per_call = 6 * (K // 32) + 2 * (K // 128) + 3
     elif kind == "gridnoise":
         N, K, b = vals
         W = synth.weights_torch(N, K, device=dev)

@@ -371,7 +371,7 @@ slq_status slq_grid_noise(const void *W_bf16, int64_t N, int64_t K, int bits,
  * flags      device uint32 or NULL: SLQ_FLAG_NONFINITE, _SCALE_OVERFLOW as
  *            for slq_quantize; SLQ_FLAG_NOT_POSITIVE_DEFINITE when the damped
  *            H (or its inverse) has a non-positive Cholesky pivot.
- * Runs about 2 K + 2 K/128 + 8 launches on `stream`.  Errors:
+ * Runs 6 K/32 + 2 K/128 + 3 launches on `stream`.  Errors:
  * SLQ_ERR_INVALID_ARGUMENT for sizes, alignment, a short workspace or
  * overlapping buffers, before any launch; SLQ_ERR_CUDA for a failed launch.
  */

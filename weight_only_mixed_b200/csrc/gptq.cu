@@ -24,16 +24,18 @@
 // the blocked column updates apply a block's 128 terms to every later column
 // in column order, exactly as the column-by-column definition does.  The
 // codes, scales and zeros are therefore the definition's own, bit for bit,
-// whatever the launch shape.  Parallelism comes from independent elements:
-// (i, j) pairs of H and H^-1, rows of a Cholesky column, columns of the
-// triangular inverse, rows of W, and (row, column) pairs of each trailing
-// update.
+// whatever the launch shape.  The factorizations run right-looking in blocks
+// of 32: a block is finished by one CTA, and the updates it owes every later
+// element are applied by a parallel trailing kernel, each element walking the
+// block's columns (or rows) in order -- the same subtractions, in the same
+// order, as the left-looking definition.  Parallelism comes from independent
+// elements: (i, j) pairs of H and H^-1, the trailing elements of each block,
+// rows of W, and (row, column) pairs of each group's trailing update.
 //
 // Storage (binary64 workspace): Hm holds H, then its lower Cholesky factor
 // column-major (element (i, k) at Hm[k K + i]), then H^-1, then the factor of
-// H^-1, i.e. U^T (U_kj at Hm[k K + j]); Lr holds L row-major, then the
-// inverse's columns transposed; Dg holds the inverse along diagonals
-// (Dg[s K + c] = (L^-1)[c + s][c]), the access order of its column sweeps.
+// H^-1, i.e. U^T (U_kj at Hm[k K + j]); Dg holds Z = L^-1 row-major; Lr holds
+// Z transposed.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -109,78 +111,160 @@ __global__ void damp_kernel(double* __restrict__ H, int K, double damp, const do
 }
 
 // ---------------------------------------------------------------------------
-// Lower Cholesky factor, left-looking, one launch per column j (A symmetric,
-// read column-major; column j of L overwrites column j):
-//   d = a_jj - sum_{k<j} L_jk^2;  L_jj = sqrt(d);
-//   L_ij = (a_ij - sum_{k<j} L_ik L_jk) / L_jj   (i > j).
-// Every thread forms d itself (the same operations, so the same value).
+// Lower Cholesky factor, A symmetric and column-major (element (i, j) at
+// A[j K + i]), overwritten by L.  The definition, per element:
+//   d_j = a_jj - sum_{k<j} L_jk L_jk;  L_jj = sqrt(d_j);
+//   L_ij = (a_ij - sum_{k<j} L_ik L_jk) / L_jj          (i > j, k ascending).
+// Right-looking blocked form with the same per-element sequence: once column
+// k is final, every later element (i, j) has L_ik L_jk subtracted, in k order
+// -- inside a 32-column panel by one CTA, below and to the right of it by the
+// trailing kernel, each element walking the panel's columns in order.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) chol_col_kernel(double* __restrict__ A, int K, int j,
-                                                       uint32_t* __restrict__ flags) {
-  const int i = j + blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= K) return;
-  const double* colj = A;  // element (r, k) at A[k K + r]
-  double d = A[static_cast<int64_t>(j) * K + j];
-  double v = A[static_cast<int64_t>(j) * K + i];
-  // Unrolled so that the loads of several steps are in flight: the chains
-  // themselves (d and v, in k order) are unchanged.
-#pragma unroll 8
-  for (int k = 0; k < j; ++k) {
-    const double ljk = colj[static_cast<int64_t>(k) * K + j];
-    d = __dsub_rn(d, __dmul_rn(ljk, ljk));
-    v = __dsub_rn(v, __dmul_rn(colj[static_cast<int64_t>(k) * K + i], ljk));
+constexpr int kP = 32;  // panel width (rows of a triangular-inverse block)
+
+__global__ void __launch_bounds__(1024) chol_panel_kernel(double* __restrict__ A, int K, int p0,
+                                                          uint32_t* __restrict__ flags) {
+  __shared__ double dsh;
+  const int pend = p0 + kP;
+  for (int j = p0; j < pend; ++j) {
+    double* colj = A + static_cast<int64_t>(j) * K;
+    if (threadIdx.x == 0) {
+      double d = colj[j];
+      if (!(d > 0.0)) {
+        if (flags) atomicOr(flags, kFlagNotPositiveDefinite);
+        d = 1.0;  // keep going; the outputs are flagged as unspecified
+      }
+      d = __dsqrt_rn(d);
+      colj[j] = d;
+      dsh = d;
+    }
+    __syncthreads();
+    const double d = dsh;
+    for (int i = j + 1 + threadIdx.x; i < K; i += blockDim.x) colj[i] = __ddiv_rn(colj[i], d);
+    __syncthreads();
+    // The panel's later columns j' (and rows i >= j'): a_ij' -= L_ij L_j'j.
+    const int ncol = pend - j - 1;
+    if (ncol > 0) {
+      const int64_t rows = K - (j + 1);
+      for (int64_t idx = threadIdx.x; idx < rows * ncol; idx += blockDim.x) {
+        const int jp = j + 1 + static_cast<int>(idx % ncol);
+        const int i = j + 1 + static_cast<int>(idx / ncol);
+        if (i >= jp) {
+          double& a = A[static_cast<int64_t>(jp) * K + i];
+          a = __dsub_rn(a, __dmul_rn(colj[i], colj[jp]));
+        }
+      }
+    }
+    __syncthreads();
   }
-  if (!(d > 0.0)) {
-    if (i == j && flags) atomicOr(flags, kFlagNotPositiveDefinite);
-    d = 1.0;  // keep going; the outputs are flagged as unspecified
-  }
-  d = __dsqrt_rn(d);
-  A[static_cast<int64_t>(j) * K + i] = i == j ? d : __ddiv_rn(v, d);
 }
 
-// Lr[i][k] = L_ik (row-major, zero above the diagonal) from the column-major factor.
-__global__ void __launch_bounds__(256) lower_to_rows_kernel(const double* __restrict__ A, int K,
-                                                            double* __restrict__ Lr) {
+// Elements (i, j) with j >= p0 + 32, i >= j: a_ij -= L_ik L_jk for the
+// panel's k in order.  64 x 64 tiles of the lower triangle.
+constexpr int kC = 64;
+__global__ void __launch_bounds__(256) chol_trailing_kernel(double* __restrict__ A, int K, int p0) {
+  const int q0 = p0 + kP;
+  const int bi = blockIdx.y, bj = blockIdx.x;
+  if (bj > bi) return;
+  const int i0 = q0 + bi * kC, j0 = q0 + bj * kC;
+  __shared__ double li[kP][kC + 1], lj[kP][kC + 1];  // [k][row]
+  for (int idx = threadIdx.x; idx < kP * kC; idx += blockDim.x) {
+    const int k = idx / kC, r = idx % kC;
+    const double* col = A + static_cast<int64_t>(p0 + k) * K;
+    li[k][r] = i0 + r < K ? col[i0 + r] : 0.0;
+    lj[k][r] = j0 + r < K ? col[j0 + r] : 0.0;
+  }
+  __syncthreads();
+  const int r = threadIdx.x % kC, c0 = threadIdx.x / kC;  // row r, columns c0 + 4 e
+  const int i = i0 + r;
+  if (i >= K) return;
+#pragma unroll 4
+  for (int e = 0; e < kC / 4; ++e) {
+    const int c = c0 + 4 * e, j = j0 + c;
+    if (j >= K || j > i) continue;
+    double& a = A[static_cast<int64_t>(j) * K + i];
+    double v = a;
+    for (int k = 0; k < kP; ++k) v = __dsub_rn(v, __dmul_rn(li[k][r], lj[k][c]));
+    a = v;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Z = L^-1, row-major V (V[i][c] = Z_ic once row i is final).  The
+// definition, per element: Z_ic = (delta_ic - sum_{k=c}^{i-1} L_ik Z_kc) /
+// L_ii, k ascending.  Right-looking by rows with the same sequence: V starts
+// as the identity; once row k is final, every later row i has L_ik Z_kc
+// subtracted from V[i][c] for c <= k -- inside a block of 32 rows by one
+// CTA, below it by the trailing kernel, each element walking the block's
+// rows in order.  L is read from the column-major factor.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) identity_kernel(double* __restrict__ V, int K) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx < static_cast<int64_t>(K) * K) V[idx] = (idx / K == idx % K) ? 1.0 : 0.0;
+}
+
+__global__ void __launch_bounds__(1024) inv_block_kernel(const double* __restrict__ L, int K, int r0,
+                                                         double* __restrict__ V) {
+  const int rend = r0 + kP;
+  for (int i = r0; i < rend; ++i) {
+    double* vi = V + static_cast<int64_t>(i) * K;
+    const double lii = L[static_cast<int64_t>(i) * K + i];
+    for (int c = threadIdx.x; c <= i; c += blockDim.x) vi[c] = __ddiv_rn(vi[c], lii);
+    __syncthreads();
+    // The block's later rows i' (columns c <= i): v_i'c -= L_i'i Z_ic.
+    const int nrow = rend - i - 1;
+    if (nrow > 0) {
+      const int64_t cols = i + 1;
+      for (int64_t idx = threadIdx.x; idx < cols * nrow; idx += blockDim.x) {
+        const int ip = i + 1 + static_cast<int>(idx / cols);
+        const int c = static_cast<int>(idx % cols);
+        double& v = V[static_cast<int64_t>(ip) * K + c];
+        v = __dsub_rn(v, __dmul_rn(L[static_cast<int64_t>(i) * K + ip], vi[c]));
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// Rows i' >= r0 + 32, columns c < r0 + 32: v_i'c -= L_i'k Z_kc for the
+// block's rows k >= c, in order.  64 x 64 tiles.
+__global__ void __launch_bounds__(256) inv_trailing_kernel(const double* __restrict__ L, int K, int r0,
+                                                           double* __restrict__ V) {
+  const int i0 = r0 + kP + blockIdx.y * kC, c0 = blockIdx.x * kC;
+  __shared__ double lk[kP][kC + 1], zk[kP][kC + 1];  // [k][row i'], [k][column c]
+  for (int idx = threadIdx.x; idx < kP * kC; idx += blockDim.x) {
+    const int k = idx / kC, r = idx % kC;
+    lk[k][r] = i0 + r < K ? L[static_cast<int64_t>(r0 + k) * K + i0 + r] : 0.0;  // L_{i0+r, r0+k}
+    zk[k][r] = c0 + r < r0 + kP ? V[static_cast<int64_t>(r0 + k) * K + c0 + r] : 0.0;
+  }
+  __syncthreads();
+  const int c = threadIdx.x % kC, rr = threadIdx.x / kC;  // column c, rows rr + 4 e
+  const int cg = c0 + c;
+  if (cg >= r0 + kP) return;
+  const int kstart = cg > r0 ? cg - r0 : 0;  // the block's rows k >= c
+#pragma unroll 4
+  for (int e = 0; e < kC / 4; ++e) {
+    const int ip = i0 + rr + 4 * e;
+    if (ip >= K) continue;
+    double& a = V[static_cast<int64_t>(ip) * K + cg];
+    double v = a;
+    for (int k = kstart; k < kP; ++k) v = __dsub_rn(v, __dmul_rn(lk[k][rr + 4 * e], zk[k][c]));
+    a = v;
+  }
+}
+
+// ZT[i][k] = Z_ki from the row-major V (a tiled transpose; zero above).
+__global__ void __launch_bounds__(256) transpose_kernel(const double* __restrict__ V, int K,
+                                                        double* __restrict__ ZT) {
   __shared__ double tile[kT][kT + 1];
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  const int k0 = blockIdx.x * kT, i0 = blockIdx.y * kT;
-  for (int r = ty; r < kT; r += 8) tile[r][tx] = A[static_cast<int64_t>(k0 + r) * K + i0 + tx];  // (i0+tx, k0+r)
+  const int c0 = blockIdx.x * kT, k0 = blockIdx.y * kT;
+  for (int r = ty; r < kT; r += 8) tile[r][tx] = V[static_cast<int64_t>(k0 + r) * K + c0 + tx];  // Z_{k0+r, c0+tx}
   __syncthreads();
   for (int r = ty; r < kT; r += 8) {
-    const int i = i0 + r, k = k0 + tx;
-    Lr[static_cast<int64_t>(i) * K + k] = k <= i ? tile[tx][r] : 0.0;
+    const int i = c0 + r, k = k0 + tx;
+    ZT[static_cast<int64_t>(i) * K + k] = k >= i ? tile[tx][r] : 0.0;
   }
-}
-
-// ---------------------------------------------------------------------------
-// Z = L^-1 by forward substitution, one thread per column c:
-//   Z_ic = (delta_ic - sum_{k=c}^{i-1} L_ik Z_kc) / L_ii   (i >= c).
-// Stored along diagonals, Dg[s K + c] = Z_{c+s, c}, so that the threads of a
-// warp read consecutive addresses.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) tri_inverse_kernel(const double* __restrict__ Lr, int K,
-                                                          double* __restrict__ Dg) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  const int c0 = blockIdx.x * blockDim.x;  // the warp walks rows together from its first column
-  if (c >= K) return;
-  for (int i = c0; i < K; ++i) {
-    if (i < c) continue;
-    const double* li = Lr + static_cast<int64_t>(i) * K + c;  // L_{i, c + s}
-    double v = i == c ? 1.0 : 0.0;
-    const int n = i - c;
-#pragma unroll 8
-    for (int s = 0; s < n; ++s) v = __dsub_rn(v, __dmul_rn(li[s], Dg[static_cast<int64_t>(s) * K + c]));
-    Dg[static_cast<int64_t>(n) * K + c] = __ddiv_rn(v, Lr[static_cast<int64_t>(i) * K + i]);
-  }
-}
-
-// ZT[i][k] = Z_ki (zero for k < i) from the diagonal storage.
-__global__ void __launch_bounds__(256) diag_to_rows_kernel(const double* __restrict__ Dg, int K,
-                                                           double* __restrict__ ZT) {
-  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= static_cast<int64_t>(K) * K) return;
-  const int i = static_cast<int>(idx / K), k = static_cast<int>(idx % K);
-  ZT[idx] = k >= i ? Dg[static_cast<int64_t>(k - i) * K + i] : 0.0;
 }
 
 // H^-1 = Z^T Z: (H^-1)_ij = sum_{k >= max(i, j)} Z_ki Z_kj, ascending k.  The
@@ -406,8 +490,25 @@ Ws carve(void* base, int64_t N, int64_t K) {
 }
 
 cudaError_t cholesky(double* A, int K, uint32_t* flags, cudaStream_t stream) {
-  for (int j = 0; j < K; ++j) {
-    chol_col_kernel<<<(K - j + 255) / 256, 256, 0, stream>>>(A, K, j, flags);
+  for (int p0 = 0; p0 < K; p0 += kP) {
+    chol_panel_kernel<<<1, 1024, 0, stream>>>(A, K, p0, flags);
+    const int rest = K - p0 - kP;
+    if (rest > 0) {
+      const int t = (rest + kC - 1) / kC;
+      chol_trailing_kernel<<<dim3(t, t), 256, 0, stream>>>(A, K, p0);
+    }
+  }
+  return cudaGetLastError();
+}
+
+// Z = L^-1 into V (row-major), L column-major.
+cudaError_t tri_inverse(const double* L, int K, double* V, cudaStream_t stream) {
+  identity_kernel<<<static_cast<unsigned>((static_cast<int64_t>(K) * K + 255) / 256), 256, 0, stream>>>(V, K);
+  for (int r0 = 0; r0 < K; r0 += kP) {
+    inv_block_kernel<<<1, 1024, 0, stream>>>(L, K, r0, V);
+    const int rest = K - r0 - kP;
+    if (rest > 0)
+      inv_trailing_kernel<<<dim3((r0 + kP + kC - 1) / kC, (rest + kC - 1) / kC), 256, 0, stream>>>(L, K, r0, V);
   }
   return cudaGetLastError();
 }
@@ -430,9 +531,9 @@ cudaError_t launch_gptq(const uint16_t* W, int64_t N, int64_t K, int bits, const
   damp_kernel<<<(k + 255) / 256, 256, 0, stream>>>(ws.hm, k, damp, ws.mean);
   cudaError_t e = cholesky(ws.hm, k, flags, stream);
   if (e != cudaSuccess) return e;
-  lower_to_rows_kernel<<<tiles, 256, 0, stream>>>(ws.hm, k, ws.lr);
-  tri_inverse_kernel<<<(k + 127) / 128, 128, 0, stream>>>(ws.lr, k, ws.dg);
-  diag_to_rows_kernel<<<static_cast<unsigned>((K * K + 255) / 256), 256, 0, stream>>>(ws.dg, k, ws.lr);
+  e = tri_inverse(ws.hm, k, ws.dg, stream);
+  if (e != cudaSuccess) return e;
+  transpose_kernel<<<tiles, 256, 0, stream>>>(ws.dg, k, ws.lr);
   inverse_product_kernel<<<tiles, 256, 0, stream>>>(ws.lr, k, ws.hm);
   e = cholesky(ws.hm, k, flags, stream);  // U^T, column-major: U_kj at hm[k K + j]
   if (e != cudaSuccess) return e;
