@@ -51,6 +51,30 @@ __device__ __forceinline__ void load_unit(const uint8_t* st, int row, int u, uin
   }
 }
 
+// 2b words (64 codes: units 2h and 2h + 1) of row `row` of a stage, with the
+// widest loads the row's alignment allows: when the 32 lanes of a warp read
+// 32 consecutive rows, b = 2, 4, 8 are conflict free and the other widths
+// at most two-way conflicted.
+template <int B>
+__device__ __forceinline__ void load_half(const uint8_t* st, int row, int h, uint32_t (&w)[2][B]) {
+  uint32_t* f = &w[0][0];
+  if constexpr (B == 8 || B == 4 || B == 2 || B == 6) {
+    const uint32_t off = row * 16 * B + 8 * B * h;  // 16-byte aligned
+#pragma unroll
+    for (int i = 0; i < B / 2; ++i) {
+      const uint4 v = *reinterpret_cast<const uint4*>(st + p_swz<B>(off + 16 * i));
+      f[4 * i] = v.x; f[4 * i + 1] = v.y; f[4 * i + 2] = v.z; f[4 * i + 3] = v.w;
+    }
+  } else {
+    const uint2* p = reinterpret_cast<const uint2*>(st + row * 16 * B + 8 * B * h);  // 8-byte aligned
+#pragma unroll
+    for (int i = 0; i < B; ++i) {
+      const uint2 v = p[i];
+      f[2 * i] = v.x; f[2 * i + 1] = v.y;
+    }
+  }
+}
+
 template <int B>
 __device__ __forceinline__ uint32_t code_at(const uint32_t (&w)[B], int i) {
   const int o = B * i;
