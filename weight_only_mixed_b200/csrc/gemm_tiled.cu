@@ -468,9 +468,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 // and two A buffers of 64 columns (128 codes per row, two bf16 per column)
 // at 384 and 448.
 //
-// The activation ring holds whole groups: slot s = g % kXG takes the two
-// 64-k stages of group g on one barrier; gdone[s] (one commit per MMA
-// stream) frees both that slot and A buffer g % 2.
+// Each issuing thread waits on two barriers and commits once per group
+// (a second commit per group was measured to cost ~15 % of the tensor
+// core's time): ready[s] completes when group g's activations have landed
+// (slot s = g % kXG of the activation ring, both 64-k stages) and its A tile
+// is in TMEM; pe[b] when product buffer b is free.  Its commit goes to
+// gdone[s], which completes once every stream's products of group g are
+// done: the fold warps wait on it, and it frees activation slot s and A
+// buffer g % 2.
 //
 // Warp roles (768 threads, one CTA per SM):
 //   warp 0        TMA producer of X (two 64 k x BN tiles per group).
@@ -548,19 +553,20 @@ __global__ void __maxnreg__(kRegsTm)
   uint16_t* sring = reinterpret_cast<uint16_t*>(pbuf + kSP * p_stage_bytes<B>());  // [kSRing][128]
   uint8_t* zring = reinterpret_cast<uint8_t*>(sring + kSRing * kBM);                // [kSRing][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(zring + kSRing * kBM);
-  // x_full[kXG], gdone[kXG], a_full[2], p_full[kSP], p_empty[kSP], pf[3], pe[3], mma_done
+  // ready[kXG], gdone[kXG], p_full[kSP], p_empty[kSP], pf[3], pe[3], mma_done
   Bars sh;
-  sh.x_full = bars;
-  sh.x_empty = sh.x_full + kXG;  // gdone: the group's MMAs (both streams) completed
-  sh.a_full = sh.x_empty + kXG;
+  sh.x_full = bars;              // ready: group's X landed and its A tile written
+  sh.x_empty = sh.x_full + kXG;  // gdone: the group's products complete
+  sh.a_full = nullptr;
   sh.a_empty = nullptr;
-  sh.p_full = sh.a_full + 2;
+  sh.p_full = sh.x_empty + kXG;
   sh.p_empty = sh.p_full + kSP;
   sh.pf = sh.p_empty + kSP;
   sh.pe = sh.pf + kPBufs;
   sh.mma_done = sh.pe + kPBufs;
   sh.tmem_base = reinterpret_cast<uint32_t*>(sh.mma_done + 1);
   sh.abort_flag = reinterpret_cast<volatile int*>(sh.tmem_base + 1);
+  uint64_t* ready = sh.x_full;
   uint64_t* gdone = sh.x_empty;
 
   const int warp = threadIdx.x >> 5;
@@ -575,10 +581,9 @@ __global__ void __maxnreg__(kRegsTm)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kXG; ++i) {
-      mbar_init(&sh.x_full[i], 1);
+      mbar_init(&ready[i], 1 + kUnpackWarpsTm);  // X producer (expect_tx) + unpack warps
       mbar_init(&gdone[i], kNH);  // one commit per MMA stream
     }
-    for (int i = 0; i < 2; ++i) mbar_init(&sh.a_full[i], kUnpackWarpsTm);
     for (int i = 0; i < kSP; ++i) {
       mbar_init(&sh.p_full[i], 1 + 32);  // TMA arrival + the producer warp's lanes
       mbar_init(&sh.p_empty[i], kUnpackWarpsTm);
@@ -620,15 +625,15 @@ __global__ void __maxnreg__(kRegsTm)
         for (int g = 0; g < ng; ++g) {
           const int s = g % kXG;
           if (g >= kXG && !wait_or_abort(&gdone[s], ((g / kXG) - 1) & 1, sh, flags)) break;
-          mbar_arrive_expect_tx(&sh.x_full[s], kSlot);
-          tma_load_2d(xbuf + s * kSlot, &tmap_x, &sh.x_full[s], (2 * (g_begin + g)) * kBK, m0);
-          tma_load_2d(xbuf + s * kSlot + C::kXStage, &tmap_x, &sh.x_full[s],
+          mbar_arrive_expect_tx(&ready[s], kSlot);
+          tma_load_2d(xbuf + s * kSlot, &tmap_x, &ready[s], (2 * (g_begin + g)) * kBK, m0);
+          tma_load_2d(xbuf + s * kSlot + C::kXStage, &tmap_x, &ready[s],
                       (2 * (g_begin + g) + 1) * kBK, m0);
           ++issued;
         }
         // Drain: every issued copy must land before the CTA may exit.
         for (int i = issued - kXG; i < issued; ++i)
-          if (i >= 0) mbar_wait_bounded(&sh.x_full[i % kXG], (i / kXG) & 1);
+          if (i >= 0) mbar_wait_bounded(&ready[i % kXG], (i / kXG) & 1);
       }
       __syncwarp();
     } else if (warp == kWarpW) {
@@ -690,8 +695,7 @@ __global__ void __maxnreg__(kRegsTm)
           const int a = g & 1, s = g % kXG;
           const int h = kNH * g + j;
           const int pb = h % kPBufs;
-          ok = wait_or_abort(&sh.a_full[a], (g >> 1) & 1, sh, flags) &&
-               wait_or_abort(&sh.x_full[s], (g / kXG) & 1, sh, flags) &&
+          ok = wait_or_abort(&ready[s], (g / kXG) & 1, sh, flags) &&
                wait_or_abort(&sh.pe[pb], ((h / kPBufs) & 1) ^ 1, sh, flags);
           if (!ok) break;
           tc_fence_after_sync();
@@ -705,7 +709,6 @@ __global__ void __maxnreg__(kRegsTm)
             const uint64_t db = (kk < 4 ? db0 : db1) + 2 * (kk & 3);
             umma_bf16_ts(d, at + static_cast<uint32_t>(8 * kk), db, idesc, kk > 0 ? 1u : 0u);
           }
-          umma_commit(&sh.pf[pb]);
           umma_commit(&gdone[s]);
         }
         umma_commit(sh.mma_done);
@@ -747,7 +750,7 @@ __global__ void __maxnreg__(kRegsTm)
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&sh.a_full[a]);
+        mbar_arrive(&ready[g % kXG]);
         mbar_arrive(&sh.p_empty[sp]);
       }
     }
@@ -769,7 +772,7 @@ __global__ void __maxnreg__(kRegsTm)
     for (int g = 0; g < ng && ok; ++g) {
       const int h = kNH * g + jh;
       const int pb = h % kPBufs;
-      ok = __all_sync(0xffffffffu, wait_or_abort(&sh.pf[pb], (h / kPBufs) & 1, sh, flags));
+      ok = __all_sync(0xffffffffu, wait_or_abort(&gdone[g % kXG], (g / kXG) & 1, sh, flags));
       if (!ok) break;
       tc_fence_after_sync();
       const float s = __half2float(__ushort_as_half(sring[(g % kSRing) * kBM + row]));
