@@ -158,6 +158,38 @@ def gemm(x_bf16, packed, scales, zeros, K: int, bits: int, rows=None) -> np.ndar
     return y
 
 
+def bf16_rn(values) -> np.ndarray:
+    """bf16 bits of binary64 values that binary32 holds exactly, rounded to
+    nearest, ties to even (the rounding of IEEE-754 conversions)."""
+    v = np.asarray(values, dtype=np.float64)
+    f = v.astype(np.float32)
+    if not np.array_equal(f.astype(np.float64), v, equal_nan=True):
+        raise ValueError("bf16_rn expects values exact in binary32")
+    u = f.view(np.uint32).astype(np.uint64)
+    r = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return r.astype(np.uint16)
+
+
+def fake_quant_bf16(packed, scales, zeros, K: int, bits: int) -> np.ndarray:
+    """The layer's bf16 fake-quantized weights, [N, K] bf16 bits:
+    bf16_rn(s * (q - z)) per weight -- the form in which the exported
+    checkpoints store the quantized layer (GitHub README, "Export").  The
+    product s * (q - z) is exact in binary64 and in binary32 (11 + 8
+    significant bits), so the rounding to bf16 is the only one."""
+    return bf16_rn(dequantize(packed, scales, zeros, K, bits))
+
+
+def gemm_fake_quant(x_bf16, packed, scales, zeros, K: int, bits: int, rows=None) -> np.ndarray:
+    """y = X[rows] W_bf16^T in binary64, W_bf16 = fake_quant_bf16(...)."""
+    x = _u16(x_bf16)
+    if rows is not None:
+        x = x[np.asarray(rows, dtype=np.int64)]
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    w = fake_quant_bf16(packed, scales, zeros, K, bits)
+    wf = (w.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return xf @ wf.T
+
+
 def ear_kl(a_bf16, b_bf16, tau: float, rows=None):
     """Per-token (EAR, KL) in binary64 for the selected rows."""
     a = _u16(a_bf16)
