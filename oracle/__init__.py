@@ -173,7 +173,8 @@ def bf16_rn(values) -> np.ndarray:
 def fake_quant_bf16(packed, scales, zeros, K: int, bits: int) -> np.ndarray:
     """The layer's bf16 fake-quantized weights, [N, K] bf16 bits:
     bf16_rn(s * (q - z)) per weight -- the form in which the exported
-    checkpoints store the quantized layer (GitHub README, "Export").  The
+    checkpoints store the quantized layer (GitHub README, "4. Build and
+    serve a checkpoint").  The
     product s * (q - z) is exact in binary64 and in binary32 (11 + 8
     significant bits), so the rounding to bf16 is the only one."""
     return bf16_rn(dequantize(packed, scales, zeros, K, bits))

@@ -12,9 +12,10 @@
 //
 // Weights.  Each code is dequantized to bf16_rn(s * (q - z)): the exact
 // binary32 product rounded once to bf16, i.e. the weight of the layer's bf16
-// fake-quantized copy (the pages' checkpoint format; GitHub README,
-// "Export").  With the scale inside the weight, one TMEM accumulator runs
-// over the whole K range and no per-group rescaling is needed.
+// fake-quantized copy (the form in which the pages' checkpoints store a
+// quantized layer; GitHub README, "4. Build and serve a checkpoint").  With
+// the scale inside the weight, one TMEM accumulator runs over the whole K
+// range and no per-group rescaling is needed.
 //
 // Where the time goes, per 128-wide group of a 128 x 256 tile (1024 clocks
 // of tensor-core work):
