@@ -147,6 +147,21 @@ __device__ __forceinline__ void unit_pairs(const uint32_t (&w)[B], uint32_t z, u
 template <int B>
 __device__ __forceinline__ void unit_scaled(const uint32_t (&w)[B], uint32_t z, float s,
                                             uint32_t (&out)[16]) {
+  if constexpr (B == 8) {
+    // Bytes straight into binary32 2^23 + q; (2^23 + q) - (2^23 + z) is exact.
+    const float zf = __uint_as_float(0x4B000000u | z);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float lo = __fsub_rn(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7540 | (2 * h))), zf);
+        const float hi = __fsub_rn(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7540 | (2 * h + 1))), zf);
+        __nv_bfloat162 v = __floats2bfloat162_rn(lo * s, hi * s);
+        out[2 * i + h] = *reinterpret_cast<uint32_t*>(&v);
+      }
+    }
+    return;
+  }
   unit_pairs<B>(w, z, out);
 #pragma unroll
   for (int p = 0; p < 16; ++p) {
