@@ -549,7 +549,15 @@ __global__ void __launch_bounds__(kThreads)
 // the register lists), and K lanes form the terms.
 // ---------------------------------------------------------------------------
 constexpr int kTopMax = 16;
-constexpr int kTopThreads = 512;
+// Small CTAs, several per SM: a CTA's end-of-row merge (warp 0 alone, the
+// others at the barrier) then overlaps the other CTAs' streaming.  One
+// 512-thread CTA per SM (~100 registers a thread) left the SM idle during
+// every merge.  On 4096 x 151936, K = 10: 1089 us with 512 threads (1 CTA
+// per SM), 635 with 128 (4 per SM), 573 with 64 (8 per SM); with fewer rows
+// than 2 per 64-thread CTA the 128-thread shape is faster (T = 512: 98
+// against 130 us).
+constexpr int kTopThreadsSmall = 64, kTopCtasSmall = 8;
+constexpr int kTopThreadsLarge = 128, kTopCtasLarge = 4;
 
 // (v, i) ranks before (w, j): larger logit first, lower index on ties.
 __device__ __forceinline__ bool top_before(float v, int i, float w, int j) {
@@ -658,7 +666,7 @@ __device__ __forceinline__ float warp_kth_largest(float m, int K) {
   return __shfl_sync(kFull, m, K - 1);
 }
 
-template <bool kVec, int KM>
+template <bool kVec, int KM, int kTopThreads>
 __global__ void __launch_bounds__(kTopThreads)
     ear_kl_topk_kernel(const uint16_t* __restrict__ A, const uint16_t* __restrict__ Bq, int64_t T,
                        int64_t V, int K, float c, float* __restrict__ ear_tok,
@@ -881,16 +889,22 @@ cudaError_t launch_ear_kl_topk(const uint16_t* a, const uint16_t* b, int64_t T, 
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const float c = 1.4426950408889634f / temperature;
-  const int64_t cap = 2 * static_cast<int64_t>(sms);
+  const bool small = T >= 2 * kTopCtasSmall * static_cast<int64_t>(sms);
+  const int64_t cap = (small ? kTopCtasSmall : kTopCtasLarge) * static_cast<int64_t>(sms);
   const unsigned blocks = static_cast<unsigned>(T < cap ? T : cap);
   const bool aligned = ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b)) & 15u) == 0;
   const bool vec = V % 8 == 0 && aligned;
   auto run = [&](auto km) {
     constexpr int KM = decltype(km)::value;
-    if (vec)
-      ear_kl_topk_kernel<true, KM><<<blocks, kTopThreads, 0, stream>>>(a, b, T, V, K, c, ear_tok, kl_tok);
+    constexpr int NS = kTopThreadsSmall, NL = kTopThreadsLarge;
+    if (vec && small)
+      ear_kl_topk_kernel<true, KM, NS><<<blocks, NS, 0, stream>>>(a, b, T, V, K, c, ear_tok, kl_tok);
+    else if (vec)
+      ear_kl_topk_kernel<true, KM, NL><<<blocks, NL, 0, stream>>>(a, b, T, V, K, c, ear_tok, kl_tok);
+    else if (small)
+      ear_kl_topk_kernel<false, KM, NS><<<blocks, NS, 0, stream>>>(a, b, T, V, K, c, ear_tok, kl_tok);
     else
-      ear_kl_topk_kernel<false, KM><<<blocks, kTopThreads, 0, stream>>>(a, b, T, V, K, c, ear_tok, kl_tok);
+      ear_kl_topk_kernel<false, KM, NL><<<blocks, NL, 0, stream>>>(a, b, T, V, K, c, ear_tok, kl_tok);
   };
   if (K <= 1) run(std::integral_constant<int, 1>{});
   else if (K <= 2) run(std::integral_constant<int, 2>{});
