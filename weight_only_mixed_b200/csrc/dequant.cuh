@@ -22,35 +22,6 @@ __device__ __forceinline__ uint32_t p_swz(uint32_t off) {
   else return off;
 }
 
-// b words (32 codes) of row `row`, unit u (codes [32u, 32u+32)) of a stage.
-template <int B>
-__device__ __forceinline__ void load_unit(const uint8_t* st, int row, int u, uint32_t (&w)[B]) {
-  if constexpr (B == 8) {
-    const uint32_t off = row * 128 + 32 * u;
-    const uint4 v0 = *reinterpret_cast<const uint4*>(st + p_swz<8>(off));
-    const uint4 v1 = *reinterpret_cast<const uint4*>(st + p_swz<8>(off + 16));
-    w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
-    w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
-  } else if constexpr (B == 4) {
-    const uint4 v = *reinterpret_cast<const uint4*>(st + p_swz<4>(row * 64 + 16 * u));
-    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-  } else if constexpr (B == 2) {
-    const uint2 v = *reinterpret_cast<const uint2*>(st + p_swz<2>(row * 32 + 8 * u));
-    w[0] = v.x; w[1] = v.y;
-  } else if constexpr (B == 6) {
-    const uint8_t* p = st + row * 96 + 24 * u;
-#pragma unroll
-    for (int i = 0; i < 3; ++i) {
-      const uint2 v = *reinterpret_cast<const uint2*>(p + 8 * i);
-      w[2 * i] = v.x; w[2 * i + 1] = v.y;
-    }
-  } else {
-    const uint32_t* p = reinterpret_cast<const uint32_t*>(st + row * 16 * B + 4 * B * u);
-#pragma unroll
-    for (int i = 0; i < B; ++i) w[i] = p[i];
-  }
-}
-
 // 2b words (64 codes: units 2h and 2h + 1) of row `row` of a stage, with the
 // widest loads the row's alignment allows: when the 32 lanes of a warp read
 // 32 consecutive rows, b = 2, 4, 8 are conflict free and the other widths
