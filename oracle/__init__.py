@@ -7,8 +7,9 @@ CPU-baseline/reference leg may import it; the product path
 
 The arithmetic lives in ``slq_oracle.c`` (plain C, binary32 encode decisions,
 binary64 dequantize/GEMM/EAR/KL, GPTQ error feedback and grid-noise sums);
-this module only compiles it with gcc and marshals numpy arrays through
-ctypes.
+this module compiles it with gcc and marshals numpy arrays through ctypes.
+The bf16 fake-quantized weights (``bf16_rn``, ``fake_quant_bf16``) and the
+GEMM over them (``gemm_fake_quant``) are numpy, on top of the C dequantize.
 """
 from __future__ import annotations
 
