@@ -67,6 +67,10 @@ DECODE_MS = (1, 4, 16)
 # in a decoder block run as one grouped launch (q, k, v; gate, up).
 BLOCK_LAUNCHES = ((0, 1, 2), (3,), (4, 5), (6,))
 METRIC = "W{2-8}A16 GEMM weight GB/s (% HBM peak) & TFLOP/s per b and M; EAR/KL GB/s"
+WORKLOAD = ("Qwen3-8B-shaped decoder block decode: q/o 4096x4096 b5, k/v 1024x4096 b8, "
+            "gate/up 12288x4096 b4, down 4096x12288 b4, asymmetric INT g128; "
+            "M in {1,4,16}; per M: q+k+v in one slq_gemm_group launch, o, gate+up in one, down "
+            "(12 launches per step, one CUDA graph); independent X per projection")
 
 
 def weight_bytes(N, K, bits):
@@ -459,10 +463,7 @@ def run_slq(args, rank, world, local_rank):
             "dtype": "bf16",
             "data": "synthetic (seeded skewed-Gaussian weights, N(0,1) activations; no checkpoints)",
             "config": {
-                "workload": "Qwen3-8B-shaped decoder block decode: q/o 4096x4096 b5, k/v 1024x4096 b8, "
-                            "gate/up 12288x4096 b4, down 4096x12288 b4, asymmetric INT g128; "
-                            "M in {1,4,16}; per M: q+k+v in one slq_gemm_group launch, o, gate+up in one, down "
-                            "(12 launches per step, one CUDA graph); independent X per projection",
+                "workload": WORKLOAD,
                 "block_weight_bytes": BLOCK_BYTES,
                 "bytes_per_step": 3 * BLOCK_BYTES,
                 "l2": f"inputs larger than L2: {R} rotated weight copies ({R * BLOCK_BYTES / 2**20:.0f} MiB > 126 MiB L2)",
@@ -893,7 +894,9 @@ def run_reference(args, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(span / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "Qwen3-8B-shaped decoder block decode (sampled rows)", "rows_per_layer": args.cpu_rows},
+        "config": {"workload": WORKLOAD, "block_weight_bytes": BLOCK_BYTES, "bytes_per_step": 3 * BLOCK_BYTES,
+                   "parallelism": "rank 0 alone, on the host cores",
+                   "sample": f"first {args.cpu_rows} output rows of each projection per job (rows are independent)"},
         "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
