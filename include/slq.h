@@ -55,21 +55,19 @@ enum {
   SLQ_FLAG_NOT_POSITIVE_DEFINITE = 8u /* slq_gptq: a Cholesky pivot was not positive; outputs unspecified */
 };
 
-/* GEMM kernel choice for slq_gemm_ex.  The decode kernels (DECODE, GEMV)
- * form exact bf16 values from the codes, multiply on the tensor cores with
- * fp32 accumulation, one product per 128-wide group, and apply the fp16 group
- * scale to that fp32 product.  The tiled kernel multiplies the bf16
- * fake-quantized weights bf16_rn(s (q - z)) with one fp32 accumulator over K
- * (see slq_gemm). */
+/* GEMM kernel choice for slq_gemm_ex.  Every kernel forms exact bf16 values
+ * from the codes, multiplies on the tensor cores with fp32 accumulation, one
+ * product per 128-wide group, and applies the fp16 group scale to that fp32
+ * product; they differ in how the work is split. */
 typedef enum {
   SLQ_GEMM_AUTO = 0,   /* GEMV for M <= 16, TILED above */
   SLQ_GEMM_DECODE = 1, /* M <= 16: packed weights streamed by TMA, dequantized in registers
                           into mma.sync fragments, the row tiles x groups split evenly over
                           two CTAs per SM (stream-K; needs a workspace) */
-  SLQ_GEMM_TILED = 2,  /* any M >= 1: 128 x {64, 128, 256} output tiles, weights dequantized
-                          to bf16_rn(s (q - z)) into TMEM, tcgen05.mma with A from TMEM into
-                          one TMEM accumulator over K, K split over a thread-block cluster
-                          for narrow tiles */
+  SLQ_GEMM_TILED = 2,  /* any M >= 1: 128 x {64, 128, 256} output tiles, exact bf16 (q - z)
+                          written into TMEM, tcgen05.mma with A from TMEM into per-group
+                          TMEM product buffers folded by the group scale in fp32 registers,
+                          K split over a thread-block cluster for narrow tiles */
   SLQ_GEMM_GEMV = 3    /* M <= 16: one CTA per 16- or 32-row tile whose warps split K, packed
                           weights streamed with cp.async into per-warp shared-memory rings,
                           dequantized in registers into mma.sync fragments; partial tiles
@@ -167,12 +165,6 @@ slq_status slq_quantize(const void *W_bf16, int64_t N, int64_t K, int bits,
  *
  * The kernels this call selects (SLQ_GEMM_GEMV for M <= 16, SLQ_GEMM_TILED
  * above) use no memory beyond their arguments: there is no workspace.
- *
- * Weights: the M <= 16 kernels multiply the exact s * (q - z); the tiled
- * kernel multiplies bf16_rn(s * (q - z)), the layer's bf16 fake-quantized
- * weight -- the form in which the exported checkpoints store a quantized
- * layer (GitHub README, "4. Build and serve a checkpoint") -- so its result
- * is the bf16 fake-quantized layer's output up to fp32 accumulation.
  */
 slq_status slq_gemm(const void *X_bf16, int64_t M, int64_t N, int64_t K,
                     int bits, const uint32_t *packed, const void *scales_f16,

@@ -7,9 +7,8 @@ CPU-baseline/reference leg may import it; the product path
 
 The arithmetic lives in ``slq_oracle.c`` (plain C, binary32 encode decisions,
 binary64 dequantize/GEMM/EAR/KL, GPTQ error feedback and grid-noise sums);
-this module compiles it with gcc and marshals numpy arrays through ctypes.
-The bf16 fake-quantized weights (``bf16_rn``, ``fake_quant_bf16``) and the
-GEMM over them (``gemm_fake_quant``) are numpy, on top of the C dequantize.
+this module only compiles it with gcc and marshals numpy arrays through
+ctypes.
 """
 from __future__ import annotations
 
@@ -157,39 +156,6 @@ def gemm(x_bf16, packed, scales, zeros, K: int, bits: int, rows=None) -> np.ndar
     if rc != 0:
         raise ValueError("oracle_gemm rejected its arguments")
     return y
-
-
-def bf16_rn(values) -> np.ndarray:
-    """bf16 bits of binary64 values that binary32 holds exactly, rounded to
-    nearest, ties to even (the rounding of IEEE-754 conversions)."""
-    v = np.asarray(values, dtype=np.float64)
-    f = v.astype(np.float32)
-    if not np.array_equal(f.astype(np.float64), v, equal_nan=True):
-        raise ValueError("bf16_rn expects values exact in binary32")
-    u = f.view(np.uint32).astype(np.uint64)
-    r = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    return r.astype(np.uint16)
-
-
-def fake_quant_bf16(packed, scales, zeros, K: int, bits: int) -> np.ndarray:
-    """The layer's bf16 fake-quantized weights, [N, K] bf16 bits:
-    bf16_rn(s * (q - z)) per weight -- the form in which the exported
-    checkpoints store the quantized layer (GitHub README, "4. Build and
-    serve a checkpoint").  The
-    product s * (q - z) is exact in binary64 and in binary32 (11 + 8
-    significant bits), so the rounding to bf16 is the only one."""
-    return bf16_rn(dequantize(packed, scales, zeros, K, bits))
-
-
-def gemm_fake_quant(x_bf16, packed, scales, zeros, K: int, bits: int, rows=None) -> np.ndarray:
-    """y = X[rows] W_bf16^T in binary64, W_bf16 = fake_quant_bf16(...)."""
-    x = _u16(x_bf16)
-    if rows is not None:
-        x = x[np.asarray(rows, dtype=np.int64)]
-    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    w = fake_quant_bf16(packed, scales, zeros, K, bits)
-    wf = (w.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    return xf @ wf.T
 
 
 def ear_kl(a_bf16, b_bf16, tau: float, rows=None):

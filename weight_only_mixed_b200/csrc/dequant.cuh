@@ -109,40 +109,6 @@ __device__ __forceinline__ void unit_pairs(const uint32_t (&w)[B], uint32_t z, u
   }
 }
 
-// The 32 codes of a unit as 16 bf16x2 registers holding the dequantized
-// weights rounded to bf16: bf16_rn(s * (q - z)), consecutive k.  (q - z) is
-// exact (unit_pairs), the binary32 product s * (q - z) is exact (an 11-bit
-// fp16 significand times an integer below 2^8), so the conversion to bf16 is
-// the only rounding -- the value a bf16 fake-quantized copy of the layer
-// holds.
-template <int B>
-__device__ __forceinline__ void unit_scaled(const uint32_t (&w)[B], uint32_t z, float s,
-                                            uint32_t (&out)[16]) {
-  if constexpr (B == 8) {
-    // Bytes straight into binary32 2^23 + q; (2^23 + q) - (2^23 + z) is exact.
-    const float zf = __uint_as_float(0x4B000000u | z);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const float lo = __fsub_rn(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7540 | (2 * h))), zf);
-        const float hi = __fsub_rn(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7540 | (2 * h + 1))), zf);
-        __nv_bfloat162 v = __floats2bfloat162_rn(lo * s, hi * s);
-        out[2 * i + h] = *reinterpret_cast<uint32_t*>(&v);
-      }
-    }
-    return;
-  }
-  unit_pairs<B>(w, z, out);
-#pragma unroll
-  for (int p = 0; p < 16; ++p) {
-    const float lo = __uint_as_float(out[p] << 16) * s;
-    const float hi = __uint_as_float(out[p] & 0xFFFF0000u) * s;
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    out[p] = *reinterpret_cast<uint32_t*>(&v);
-  }
-}
-
 // UMMA shared-memory descriptor: K-major, 128-byte swizzle, 8-row groups
 // 1024 bytes apart (SBO), descriptor version 1 (sm_100).
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
